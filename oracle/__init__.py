@@ -1,0 +1,13 @@
+"""fp64 CPU oracle for retrieval block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the library calls this package: only the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+import it.  It shares no code with the CUDA path; both read the same seeded
+inputs from ``retrieval_block_sparse_b200.synth`` and nothing else.
+
+Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
+invariants, library routines or brute force; see the docstring of each
+function for the passage of the pages it restates.
+"""
+from .retrieval import *  # noqa: F401,F403
+from .retrieval import __all__  # noqa: F401
