@@ -1,0 +1,238 @@
+/*
+ * rba.h -- retrieval block-sparse attention on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * Context-memory retrieval attention for long-context decoding and chunked
+ * prefill.  Past K/V is cut into fixed-size blocks; each block carries
+ * representative keys (or an embedding); a query scores the blocks, keeps the
+ * top k per KV head, and runs exact softmax attention over the sink tokens,
+ * the retrieved blocks and the local window.
+ *
+ * Sources (pages, by title and section):
+ *   [ML] "MemLong: Memory-Augmented Retrieval for Long Text Modeling"
+ *        (summary page) -- 2.2.1 fixed-size chunks, 2.2.2 memory of K-V pairs
+ *        plus representation embeddings, 2.3.2 retrieval (cosine, TopK) and
+ *        memorisation M(k, v; r^m), 2.3.3 / Figure 3 retrieval-causal
+ *        attention, 2.3.4 inference (attention window k * chunk size).
+ *   [IL] InfLLM article (Tsinghua NLP, "1024K context, 100% recall") --
+ *        "method" and "overall framework": sliding window + memory units of
+ *        contiguous tokens, represented by the tokens that received the most
+ *        attention.
+ *   [LM] "Landmark Attention: Random-Access Infinite Context Length for
+ *        Transformers" (review) -- "proposed method": one landmark key per
+ *        fixed-length block, retrieval by query-landmark similarity.
+ *   [RA] RetrievalAttention summary (arXiv 2409.10516) -- "proposed method":
+ *        every key its own unit (block size 1), retrieved by vector search.
+ *
+ * Conventions for every call:
+ *   - Every device buffer is owned by the caller.  The library never
+ *     allocates or frees device memory; calls that need scratch take a
+ *     caller-provided workspace whose size a *_workspace_size() call reports.
+ *   - Pointers marked "device" must be device pointers (cudaMalloc / torch);
+ *     "host" pointers are host memory.  All tensors are dense, row-major,
+ *     with the layout given in brackets.
+ *   - Work is asynchronous on the given stream; no call synchronises except
+ *     rba_store_check and rba_decode_step_host, which say so.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns a status and launches nothing.  Errors found on
+ *     the device (index out of range, a bounded wait that gave up) set the
+ *     store's status word, read back by rba_store_check.
+ *   - No C++ exception crosses this interface.
+ *
+ * Block / token vocabulary used below (T = tokens currently in the store):
+ *   block j            tokens [j*bs, (j+1)*bs) of one (batch, kv head)
+ *   w0                 max(T - window, 0): first token of the local window
+ *   sink               tokens [0, min(sink, w0))
+ *   candidate block    a full block whose tokens meet [sink, w0); candidates
+ *                      form the contiguous range [first_cand, first_cand+nc)
+ *   attended set       sink U retrieved blocks U window, each token once
+ *   T - nb*bs > window (a partial tail block outside the window) is rejected.
+ */
+#ifndef RBA_H_
+#define RBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RBA_OK = 0,
+  RBA_ERR_INVALID_ARG = 1,  /* bad size, pointer, mode or layout; nothing launched */
+  RBA_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. head_dim outside {64,128}) */
+  RBA_ERR_WORKSPACE = 3,    /* workspace smaller than *_workspace_size() */
+  RBA_ERR_CUDA = 4,         /* a CUDA runtime call failed */
+  RBA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (status word) */
+  RBA_ERR_BOUNDS = 6        /* a device-side index check failed (status word) */
+} rba_status;
+
+typedef enum { RBA_F32 = 0, RBA_BF16 = 1 } rba_dtype;
+
+/* How a block is represented for scoring ([ML] 2.3.2 memorisation). */
+typedef enum {
+  RBA_REP_MEAN = 0,         /* mean of the block's keys; rep pool fp32 [B][Hkv][cap_blocks][1][D] */
+  RBA_REP_TOPR_ATTN = 1,    /* [IL] method: the n_rep keys that received the most attention from a
+                               probe; rep pool dtype [B][Hkv][cap_blocks][n_rep][D], positions
+                               int32 [B][Hkv][cap_blocks][n_rep] */
+  RBA_REP_EXTERNAL = 2,     /* [LM] landmark keys given by the caller; rep pool dtype
+                               [B][Hkv][cap_blocks][n_rep][D] */
+  RBA_REP_EMBED_COSINE = 3, /* [ML] 2.2.2: L2-normalised chunk embedding; rep pool fp32
+                               [B][cap_blocks][d_ret]; scored by cosine */
+  RBA_REP_IDENTITY = 4      /* [RA]: block size 1, each key is its own representation; no rep pool */
+} rba_rep_mode;
+
+typedef struct {
+  int32_t batch;            /* B */
+  int32_t n_q_heads;        /* Hq (a multiple of n_kv_heads; q head i reads kv head i / (Hq/Hkv)) */
+  int32_t n_kv_heads;       /* Hkv */
+  int32_t head_dim;         /* D: 64 or 128 */
+  int32_t block_size;       /* bs >= 1 */
+  int32_t n_rep;            /* r: representative keys per block (1 except RBA_REP_TOPR_ATTN / EXTERNAL) */
+  int32_t d_ret;            /* embedding size (RBA_REP_EMBED_COSINE), else 0 */
+  int64_t capacity_tokens;  /* tokens per (batch, kv head) the K/V pools hold (cap_blocks = cap / bs) */
+  rba_dtype dtype;          /* storage type of q, K, V and (except fp32 pools above) rep keys */
+  rba_rep_mode mode;
+} rba_store_desc;
+
+/* Opaque: host-side description of caller-owned device pools. */
+typedef struct rba_store rba_store;
+
+/* Describe a block store ([ML] 2.2.2: memory = K-V pairs + representations).
+ *   k_pool, v_pool  device, dtype [B][Hkv][capacity_tokens][D]
+ *   rep_pool        device, layout per mode above (NULL for RBA_REP_IDENTITY)
+ *   rep_pos         device int32 [B][Hkv][cap_blocks][n_rep] for RBA_REP_TOPR_ATTN (may be
+ *                   NULL: positions are then not recorded), else ignored
+ *   status_word     device int32[4], zeroed by the caller; first error code, where, detail
+ *   out             host: receives the handle (free with rba_store_destroy)
+ * Nothing is launched.  Errors: INVALID_ARG, UNSUPPORTED. */
+rba_status rba_store_create(const rba_store_desc* desc, void* k_pool, void* v_pool,
+                            void* rep_pool, int32_t* rep_pos, int32_t* status_word,
+                            rba_store** out);
+rba_status rba_store_destroy(rba_store* store);
+
+/* Candidate range for a store holding T tokens with the given sink/window
+ * (host only; see the vocabulary above).  Errors: INVALID_ARG (tail block
+ * outside the window, negative sizes, T > capacity). */
+rba_status rba_candidates(const rba_store* store, int64_t T, int32_t sink, int32_t window,
+                          int32_t* first_cand, int32_t* n_cand);
+
+/* [ML] 2.3.2 memorisation M(k, v; r^m); [IL] method (representative tokens);
+ * [LM] proposed method (landmarks).  Writes blocks [first_block,
+ * first_block + n_blocks) of every (batch, kv head):
+ *   k_src, v_src  device dtype [B][Hkv][n_blocks*bs][D], copied into the pools; both NULL when
+ *                 the pools already hold those tokens (representations only)
+ *   aux           RBA_REP_TOPR_ATTN: probe queries, device dtype [Hkv][n_aux][D]
+ *                 RBA_REP_EXTERNAL:  landmark keys, device dtype [B][Hkv][n_blocks][n_rep][D]
+ *                 RBA_REP_EMBED_COSINE: raw embeddings, device fp32 [B][n_blocks][d_ret]
+ *                 otherwise NULL
+ *   scale         logit scale for the probe softmax (RBA_REP_TOPR_ATTN), typically 1/sqrt(D)
+ * RBA_REP_TOPR_ATTN: per probe query p, softmax over the block's bs tokens of
+ * scale * p.k_t; a token's received attention is the sum over probes; the
+ * n_rep tokens with the most (ties -> lower position) are kept in ascending
+ * position.  RBA_REP_MEAN: (1/bs) sum_t k_t.  RBA_REP_EMBED_COSINE: e/|e|.
+ * Errors: INVALID_ARG (range beyond capacity, missing aux), CUDA. */
+rba_status rba_memorize(rba_store* store, const void* k_src, const void* v_src,
+                        int64_t first_block, int32_t n_blocks, const void* aux, int32_t n_aux,
+                        float scale, cudaStream_t stream);
+
+/* Block scores ([ML] 2.3.2 cosine retrieval; [LM] query-landmark similarity;
+ * [IL] relevance against representative tokens).
+ *   dot modes: q device dtype [B][Hq][n_q][D]; for candidate c of (b, kv head h)
+ *     scores[b][h][c] = sum over the group's q heads, over the n_q rows, and over the
+ *     block's n_rep keys of q . rep  (n_q > 1: a prefill chunk shares one selection)
+ *   cosine mode: q = query embeddings, device fp32 [n_q][d_ret]; store batch must be 1;
+ *     scores[i][c] = cos(q_i, M_{first_cand + c})
+ *   scores  device fp32 [B][Hkv][nc] (dot) or [n_q][nc] (cosine)
+ *   qsum_ws device fp32 [B][Hkv][D] scratch for the summed queries (dot modes; may be NULL
+ *           when Hq/Hkv * n_q <= 64)
+ * Errors: INVALID_ARG, CUDA. */
+rba_status rba_score(const rba_store* store, const void* q, int32_t n_q, int64_t T,
+                     int32_t sink, int32_t window, float* scores, float* qsum_ws,
+                     cudaStream_t stream);
+
+/* Top-k selection ([ML] 2.3.2 z^q = TopK{Cos(r^q)}; 2.3.4 the k most relevant
+ * chunks).  For each of `rows` rows of n fp32 scores, the k best positions
+ * under (larger score first, equal scores -> lower position first; -0 == +0),
+ * written in ascending order as index_base + position.
+ *   scores  device fp32 [rows][n];  idx  device int32 [rows][k]
+ *   workspace / ws_bytes  device scratch, >= rba_topk_workspace_size(rows, n, k)
+ * NaN scores are not supported.  Errors: INVALID_ARG (k > n), WORKSPACE, CUDA. */
+rba_status rba_topk(const float* scores, int32_t rows, int32_t n, int32_t k, int32_t index_base,
+                    int32_t* idx, void* workspace, size_t ws_bytes, cudaStream_t stream);
+size_t rba_topk_workspace_size(int32_t rows, int32_t n, int32_t k);
+
+/* Decode attention, split-K with online softmax and a log-sum-exp merge of
+ * the split partials ([IL] overall framework: local window + a few memory
+ * units; [ML] 2.3.3 retrieved chunks attended without a causal mask).
+ *   q    device dtype [B][Hq][D];  idx device int32 [B][Hkv][k] ascending candidate block ids
+ *   out  device fp32 [B][Hq][D];   lse device fp32 [B][Hq] (natural log) or NULL
+ *   For q head i of kv head h = i / (Hq/Hkv):
+ *     out = sum_t softmax_t(scale * q.k_t) v_t over the attended set of (b, h).
+ *   workspace >= rba_attend_workspace_size(); its first 4 KiB must be zero before the first
+ *   call (the kernels leave it zero after each call that completes).
+ * Errors: INVALID_ARG (k > nc, T > capacity), WORKSPACE, CUDA; out-of-range idx
+ * entries are skipped and flagged as RBA_ERR_BOUNDS in the status word. */
+rba_status rba_attend(const rba_store* store, const void* q, const int32_t* idx, int32_t k,
+                      int64_t T, int32_t sink, int32_t window, float scale, float* out,
+                      float* lse, void* workspace, size_t ws_bytes, cudaStream_t stream);
+size_t rba_attend_workspace_size(const rba_store* store, int32_t k, int64_t T, int32_t sink,
+                                 int32_t window);
+
+/* Chunked prefill, retrieval-causal ([ML] 2.3.3 / Figure 3): every row of a
+ * query chunk attends bidirectionally to sink U retrieved blocks U window of
+ * the memory, and causally to the chunk's own tokens (own token i' visible to
+ * row i iff i' <= i), in one joint softmax.  Tensor-core (tcgen05) tiles.
+ *   q          device bf16 [n_chunks][Hq][chunk_len][D]
+ *   idx        device int32 [n_chunks][n_sel][k], n_sel = 1 (one selection per chunk, all
+ *              heads: cosine mode) or Hkv (one per kv head)
+ *   chunk_k/v  device bf16 [n_chunks][Hkv][chunk_len][D]
+ *   out        device fp32 [n_chunks][Hq][chunk_len][D];  lse fp32 [n_chunks][Hq][chunk_len] or NULL
+ *   The store's batch is 1 (one memory shared by all chunks) or n_chunks.
+ *   workspace >= rba_attend_prefill_workspace_size().
+ * Errors: INVALID_ARG, UNSUPPORTED (dtype other than bf16, D != 128), WORKSPACE, CUDA. */
+rba_status rba_attend_prefill(const rba_store* store, const void* q, int32_t n_chunks,
+                              int32_t chunk_len, const int32_t* idx, int32_t n_sel, int32_t k,
+                              int64_t T, int32_t sink, int32_t window, const void* chunk_k,
+                              const void* chunk_v, float scale, float* out, float* lse,
+                              void* workspace, size_t ws_bytes, cudaStream_t stream);
+size_t rba_attend_prefill_workspace_size(const rba_store* store, int32_t n_chunks,
+                                         int32_t chunk_len, int32_t n_sel, int32_t k, int64_t T,
+                                         int32_t sink, int32_t window);
+
+/* One whole decode step: rba_score (dot modes) -> rba_topk per (b, kv head)
+ * -> rba_attend, with the same definitions as those calls.
+ *   q device dtype [B][Hq][D]; idx device int32 [B][Hkv][k] (written); scores device fp32
+ *   [B][Hkv][nc] (written) or NULL; out/lse as rba_attend.
+ *   workspace >= rba_decode_step_workspace_size(); first 4 KiB zero before the first call.
+ * Errors: as the three calls. */
+rba_status rba_decode_step(const rba_store* store, const void* q, int32_t k, int64_t T,
+                           int32_t sink, int32_t window, float scale, float* scores,
+                           int32_t* idx, float* out, float* lse, void* workspace,
+                           size_t ws_bytes, cudaStream_t stream);
+size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t T,
+                                      int32_t sink, int32_t window);
+
+/* rba_decode_step from and to host memory: copies q_host (host, dtype [B][Hq][D]) into
+ * q_dev, runs the step, copies out/lse/idx back into the host buffers (any of lse_host,
+ * idx_host may be NULL), then synchronises `stream`.  q_dev, idx_dev, out_dev, lse_dev are
+ * device buffers of the sizes above.  Pinned host memory makes the copies asynchronous.
+ * Errors: as rba_decode_step, plus CUDA for the copies. */
+rba_status rba_decode_step_host(const rba_store* store, const void* q_host, void* q_dev,
+                                int32_t k, int64_t T, int32_t sink, int32_t window, float scale,
+                                int32_t* idx_dev, float* out_dev, float* lse_dev,
+                                float* out_host, float* lse_host, int32_t* idx_host,
+                                void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronises `stream`, reads the store's status word, clears it, and returns
+ * the first device-side error recorded since the last check (RBA_OK if none). */
+rba_status rba_store_check(const rba_store* store, cudaStream_t stream);
+
+const char* rba_status_string(rba_status status);
+int32_t rba_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RBA_H_ */

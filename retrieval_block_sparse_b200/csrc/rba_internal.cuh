@@ -1,0 +1,144 @@
+// Internal helpers shared by the rba kernels (device and host side).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "rba.h"
+
+struct rba_store {
+  rba_store_desc d;
+  void* k;
+  void* v;
+  void* rep;
+  int32_t* rep_pos;
+  int32_t* status;
+  int64_t cap_blocks;
+};
+
+namespace rba {
+
+// ---------------------------------------------------------------------------
+// status word: [0] first error code, [1] where, [2] detail, [3] error count
+
+enum Where : int32_t {
+  kWhereAttend = 1,
+  kWhereScore = 2,
+  kWhereTopk = 3,
+  kWhereMemorize = 4,
+  kWherePrefill = 5,
+  kWhereFused = 6,
+};
+
+__device__ __forceinline__ void report(int32_t* status, int32_t code, int32_t where,
+                                       int32_t detail) {
+  if (status == nullptr) return;
+  if (atomicCAS(status, 0, code) == 0) {
+    status[1] = where;
+    status[2] = detail;
+  }
+  atomicAdd(status + 3, 1);
+}
+
+// ---------------------------------------------------------------------------
+// element types
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static constexpr int kPerVec = 4;  // elements per 16-byte vector
+  __device__ __forceinline__ static float to_f32(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static constexpr int kPerVec = 8;
+  __device__ __forceinline__ static float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+};
+
+// 16-byte vector -> floats (exact widening)
+__device__ __forceinline__ void unpack(const uint4& u, float* f, float) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ void unpack(const uint4& u, float* f, __nv_bfloat16) {
+  f[0] = __uint_as_float(u.x << 16);
+  f[1] = __uint_as_float(u.x & 0xffff0000u);
+  f[2] = __uint_as_float(u.y << 16);
+  f[3] = __uint_as_float(u.y & 0xffff0000u);
+  f[4] = __uint_as_float(u.z << 16);
+  f[5] = __uint_as_float(u.z & 0xffff0000u);
+  f[6] = __uint_as_float(u.w << 16);
+  f[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+
+// streaming 16-byte global load (read once: do not keep in L1)
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// top-k keys: larger key = better (higher score, then lower position)
+
+__device__ __forceinline__ uint32_t ordered_f32(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0) u = 0;  // -0 == +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ uint64_t topk_key(float s, uint32_t pos) {
+  return (static_cast<uint64_t>(ordered_f32(s)) << 32) | static_cast<uint32_t>(0xffffffffu - pos);
+}
+__device__ __forceinline__ uint32_t key_pos(uint64_t key) {
+  return 0xffffffffu - static_cast<uint32_t>(key);
+}
+
+// ---------------------------------------------------------------------------
+// cp.async (16 bytes, L2 only)
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
+// ---------------------------------------------------------------------------
+// host side
+
+struct Geometry {
+  int64_t T;
+  int32_t bs;
+  int32_t sink;       // requested sink (tokens below it are not in retrieved ranges)
+  int32_t sink_end;   // min(sink, w0)
+  int64_t w0;         // first window token
+  int32_t nb;         // full blocks
+  int32_t first;      // first candidate block
+  int32_t nc;         // candidates
+};
+
+rba_status geometry(const rba_store* st, int64_t T, int32_t sink, int32_t window, Geometry* g);
+int num_sms();
+
+#define RBA_CUDA_TRY(expr)                          \
+  do {                                              \
+    cudaError_t e_ = (expr);                        \
+    if (e_ != cudaSuccess) return RBA_ERR_CUDA;     \
+  } while (0)
+
+#define RBA_LAUNCH_CHECK()                          \
+  do {                                              \
+    if (cudaPeekAtLastError() != cudaSuccess) {     \
+      (void)cudaGetLastError();                     \
+      return RBA_ERR_CUDA;                          \
+    }                                               \
+  } while (0)
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline size_t dtype_size(rba_dtype t) { return t == RBA_BF16 ? 2 : 4; }
+
+}  // namespace rba

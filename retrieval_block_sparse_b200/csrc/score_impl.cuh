@@ -1,0 +1,136 @@
+// Dot-mode block scoring kernel (HBM-bound stream over representative keys).
+#pragma once
+
+#include "rba_internal.cuh"
+
+namespace rba {
+
+struct ScoreArgs {
+  const void* rep;      // [B*Hkv][rep_rows][R][D]
+  int64_t rep_rows;     // rows (blocks) per (b, kv head) in the rep pool
+  const void* q;        // [B][Hq][n_q][D] (used when qsum == nullptr)
+  const float* qsum;    // [B*Hkv][D] or nullptr
+  float* scores;        // [B*Hkv][nc]
+  int Hq, Hkv, n_q, first, nc;
+};
+
+// One CTA covers `cand_per_cta` consecutive candidates of one (b, kv head).
+// A candidate's R*D rep elements are contiguous; LPC lanes share one
+// candidate, each loading VPL 16-byte vectors, and U candidate groups are in
+// flight per warp before any arithmetic.
+template <typename QT, typename RT, int D, int R, int NW, int U>
+__global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int cand_per_cta) {
+  constexpr int EPV = Elem<RT>::kPerVec;
+  constexpr int VPC = R * D / EPV;
+  constexpr int LPC = VPC < 32 ? VPC : 32;
+  constexpr int VPL = VPC / LPC;
+  constexpr int CPW = 32 / LPC;
+  static_assert(VPC % LPC == 0 && 32 % LPC == 0, "rep row must tile the warp");
+  __shared__ float qs[D];
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hkv, h = bh - b * a.Hkv, g = a.Hq / a.Hkv;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    if (a.qsum != nullptr) {
+      acc = a.qsum[int64_t(bh) * D + d];
+    } else {
+      const QT* q = static_cast<const QT*>(a.q);
+      for (int i = 0; i < g; ++i)
+        for (int t = 0; t < a.n_q; ++t)
+          acc += Elem<QT>::to_f32(q[((int64_t(b) * a.Hq + h * g + i) * a.n_q + t) * D + d]);
+    }
+    qs[d] = acc;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % LPC, slot = lane / LPC;
+  float qr[VPL][EPV];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int d0 = ((sub + i * LPC) * EPV) % D;
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) qr[i][e] = qs[d0 + e];
+  }
+  const uint4* base = reinterpret_cast<const uint4*>(
+      static_cast<const RT*>(a.rep) + (int64_t(bh) * a.rep_rows + a.first) * (R * D));
+  const int c_begin = blockIdx.x * cand_per_cta;
+  const int c_end = min(a.nc, c_begin + cand_per_cta);
+  float* out = a.scores + int64_t(bh) * a.nc;
+  for (int c0 = c_begin + warp * CPW * U; c0 < c_end; c0 += NW * CPW * U) {
+    uint4 v[U][VPL];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * CPW + slot;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        v[u][i] = c < c_end ? ld_stream(base + int64_t(c) * VPC + sub + i * LPC)
+                            : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        float f[EPV];
+        unpack(v[u][i], f, RT());
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) acc = fmaf(qr[i][e], f[e], acc);
+      }
+#pragma unroll
+      for (int o = LPC / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      const int c = c0 + u * CPW + slot;
+      if (sub == 0 && c < c_end) out[c] = acc;
+    }
+  }
+}
+
+template <typename QT, typename RT, int D, int R>
+rba_status launch_score_dot_t(const ScoreArgs& a, int BH, cudaStream_t stream) {
+  constexpr int NW = 8, U = 4;
+  constexpr int EPV = Elem<RT>::kPerVec;
+  constexpr int VPC = R * D / EPV;
+  constexpr int LPC = VPC < 32 ? VPC : 32;
+  constexpr int per_iter = NW * (32 / LPC) * U;
+  const int64_t want = int64_t(num_sms()) * 4;
+  int64_t per_cta = (int64_t(a.nc) * BH + want - 1) / want;
+  per_cta = (per_cta + per_iter - 1) / per_iter * per_iter;
+  if (per_cta < per_iter) per_cta = per_iter;
+  const int gx = static_cast<int>((a.nc + per_cta - 1) / per_cta);
+  score_dot_kernel<QT, RT, D, R, NW, U>
+      <<<dim3(gx, BH), NW * 32, 0, stream>>>(a, static_cast<int>(per_cta));
+  RBA_LAUNCH_CHECK();
+  return RBA_OK;
+}
+
+template <typename QT, typename RT, int D>
+rba_status dispatch_r(const ScoreArgs& a, int R, int BH, cudaStream_t s) {
+  switch (R) {
+    case 1: return launch_score_dot_t<QT, RT, D, 1>(a, BH, s);
+    case 2: return launch_score_dot_t<QT, RT, D, 2>(a, BH, s);
+    case 4: return launch_score_dot_t<QT, RT, D, 4>(a, BH, s);
+    case 8: return launch_score_dot_t<QT, RT, D, 8>(a, BH, s);
+  }
+  return RBA_ERR_UNSUPPORTED;
+}
+
+template <typename QT, typename RT>
+rba_status dispatch_d(const ScoreArgs& a, int D, int R, int BH, cudaStream_t s) {
+  if (D == 128) return dispatch_r<QT, RT, 128>(a, R, BH, s);
+  if (D == 64) return dispatch_r<QT, RT, 64>(a, R, BH, s);
+  return RBA_ERR_UNSUPPORTED;
+}
+
+inline rba_status dispatch_score_dot(const ScoreArgs& a, bool q_bf16, bool rep_f32, int D, int R,
+                                     int BH, cudaStream_t s) {
+  if (q_bf16 && !rep_f32) return dispatch_d<__nv_bfloat16, __nv_bfloat16>(a, D, R, BH, s);
+  if (q_bf16 && rep_f32) return dispatch_d<__nv_bfloat16, float>(a, D, R, BH, s);
+  if (!q_bf16 && rep_f32) return dispatch_d<float, float>(a, D, R, BH, s);
+  return RBA_ERR_UNSUPPORTED;
+}
+
+rba_status launch_score_dot(const rba_store* st, const void* q, int n_q, const float* qsum,
+                            const Geometry& g, float* scores, cudaStream_t stream);
+rba_status launch_qsum(const rba_store* st, const void* q, int n_q, float* qsum,
+                       cudaStream_t stream);
+
+}  // namespace rba

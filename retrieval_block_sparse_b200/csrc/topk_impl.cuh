@@ -1,0 +1,20 @@
+// Top-k internals shared by the selector and the fused decode step.
+#pragma once
+
+#include "rba_internal.cuh"
+
+namespace rba {
+
+// Rows of at most kSmallN scores are selected by one CTA in shared memory.
+constexpr int kSmallN = 8192;
+// Largest k the radix path handles (its final sort holds k positions in smem).
+constexpr int kLargeMaxK = 16384;
+
+size_t topk_large_workspace(int rows, int n, int k);
+rba_status launch_topk_large(const float* scores, int rows, int n, int k, int index_base,
+                             int32_t* idx, void* ws, cudaStream_t stream);
+rba_status launch_topk(const float* scores, int rows, int n, int k, int index_base, int32_t* idx,
+                       void* ws, size_t ws_bytes, cudaStream_t stream);
+size_t topk_workspace(int rows, int n, int k);
+
+}  // namespace rba

@@ -1,0 +1,129 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol the header
+declares, and its host-only logic (argument checks, candidate geometry,
+workspace sizes) behaves as documented.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rba.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from retrieval_block_sparse_b200 import build
+    build.build()
+    import retrieval_block_sparse_b200 as m
+    return m.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rba_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    import retrieval_block_sparse_b200 as m
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(m.SIGNATURES), set(names) ^ set(m.SIGNATURES)
+
+
+def test_status_strings_and_version(L):
+    assert L.rba_status_string(0) == b"ok"
+    assert L.rba_status_string(3) == b"workspace too small"
+    assert L.rba_version() >= 100
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("n_rep", ctypes.c_int32),
+                ("d_ret", ctypes.c_int32), ("capacity_tokens", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("mode", ctypes.c_int32)]
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: nothing is launched
+
+
+def _create(L, **kw):
+    d = dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, block_size=16, n_rep=1, d_ret=0,
+             capacity_tokens=1024, dtype=1, mode=0)
+    d.update(kw)
+    h = ctypes.c_void_p()
+    s = L.rba_store_create(ctypes.byref(_Desc(**d)), FAKE, FAKE, FAKE, None, None,
+                           ctypes.byref(h))
+    return s, h
+
+
+def test_store_create_validates(L):
+    s, h = _create(L)
+    assert s == 0 and h.value
+    L.rba_store_destroy(h)
+    assert _create(L, head_dim=96)[0] == 2          # unsupported head dim
+    assert _create(L, n_q_heads=3)[0] == 1          # Hq not a multiple of Hkv
+    assert _create(L, mode=4)[0] == 1               # identity needs block size 1
+    assert _create(L, mode=4, block_size=1)[0] == 0
+    assert _create(L, mode=1, n_rep=17)[0] == 1     # more rep keys than tokens
+    assert _create(L, mode=3, d_ret=0)[0] == 1      # embedding size missing
+    assert _create(L, capacity_tokens=0)[0] == 1
+
+
+@pytest.mark.parametrize("T,bs,S,W", [(4096, 64, 64, 128), (131072, 128, 128, 4096),
+                                      (32768, 50, 0, 256), (1 << 20, 1, 128, 512),
+                                      (81920, 512, 0, 0), (37, 5, 3, 7), (40, 8, 8, 8),
+                                      (41, 8, 9, 2), (12, 4, 20, 0), (16, 4, 0, 16),
+                                      (100, 10, 95, 10), (50, 7, 6, 13), (0, 4, 0, 0)])
+def test_candidate_geometry_matches_oracle(L, T, bs, S, W):
+    s, h = _create(L, block_size=bs, capacity_tokens=max(T, 1) + 64,
+                   mode=4 if bs == 1 else 0)
+    assert s == 0
+    f, n = ctypes.c_int32(), ctypes.c_int32()
+    st = L.rba_candidates(h, T, S, W, ctypes.byref(f), ctypes.byref(n))
+    cand = O.candidate_blocks(T, bs, S, W)
+    if T - (T // bs) * bs > W:
+        assert st == 1
+    else:
+        assert st == 0
+        assert n.value == cand.shape[0]
+        if n.value:
+            assert f.value == cand[0]
+    L.rba_store_destroy(h)
+
+
+def test_tail_outside_window_is_rejected(L):
+    s, h = _create(L, block_size=50, capacity_tokens=40000)
+    f, n = ctypes.c_int32(), ctypes.c_int32()
+    assert L.rba_candidates(h, 32768, 0, 10, ctypes.byref(f), ctypes.byref(n)) == 1
+    assert L.rba_candidates(h, 32768, 0, 18, ctypes.byref(f), ctypes.byref(n)) == 0
+    assert L.rba_candidates(h, 50000, 0, 18, ctypes.byref(f), ctypes.byref(n)) == 1  # > capacity
+    L.rba_store_destroy(h)
+
+
+def test_host_argument_checks_launch_nothing(L):
+    s, h = _create(L)
+    # k larger than the candidate count
+    assert L.rba_attend(h, FAKE, FAKE, 1000, 1024, 0, 0, ctypes.c_float(0.1), FAKE, None, FAKE,
+                        ctypes.c_size_t(1 << 20), None) == 1
+    # workspace too small
+    assert L.rba_attend(h, FAKE, FAKE, 4, 1024, 0, 0, ctypes.c_float(0.1), FAKE, None, FAKE,
+                        ctypes.c_size_t(8), None) == 3
+    assert L.rba_topk(FAKE, 2, 10, 11, 0, FAKE, None, ctypes.c_size_t(0), None) == 1
+    assert L.rba_memorize(h, FAKE, None, 0, 1, None, 0, ctypes.c_float(1), None) == 1
+    L.rba_store_destroy(h)
+
+
+def test_workspace_sizes_are_positive(L):
+    s, h = _create(L)
+    assert L.rba_attend_workspace_size(h, 8, 1024, 16, 64) > 0
+    assert L.rba_decode_step_workspace_size(h, 8, 1024, 16, 64) > 0
+    assert L.rba_topk_workspace_size(8, 1 << 20, 2048) > 8 * (1 << 20) * 8
+    assert L.rba_topk_workspace_size(8, 1000, 32) == 0
+    L.rba_store_destroy(h)
