@@ -1,0 +1,585 @@
+#!/usr/bin/env python
+"""Decode-step throughput of retrieval block-sparse attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one whole decode step of the 128K-context GQA workload
+(infllm-decode-128k: batch 1, 32 q / 8 kv heads, head_dim 128, 131072 past
+tokens in 128-token blocks with 4 representative keys each; top-32 blocks
+per kv head + 128 sink + 4096 window tokens): block scores -> top-k ->
+split-K attention -> merge, all in librba.so.  Representations are memorised
+once before timing (memorisation is not part of a decode step).
+
+Measurement: W untimed warm-up steps, then exactly K steps replayed from CUDA
+graphs, bracketed by a barrier and a device synchronise, timed with CUDA
+events on the launching stream (max over ranks).  Steps rotate over R
+replicas of the store so that R x bytes-per-step >= 4 x L2: every step reads
+HBM, not L2.  Under torchrun each rank runs its own replica set on its own
+GPU (replicas only: the path has no exchange step), and the value is the
+total steps/s of all ranks.
+
+--impl reference times the fp64 CPU oracle on this host on bounded samples of
+the same workload (see run_reference).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "retrieval-attention decode steps/sec & achieved HBM GB/s (% roofline) at 128K ctx"
+UNIT = "steps/s"
+WORKLOAD = "infllm-decode-128k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+KERNEL_SOURCES = {
+    "attend_decode_kernel": ["csrc/attend.cu", "csrc/attend_impl.cuh", "csrc/rba_internal.cuh"],
+}
+
+
+# ---------------------------------------------------------------------------
+# plumbing
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="bound on the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, help=argparse.SUPPRESS)
+    ap.add_argument("--replicas", type=int, default=0, help=argparse.SUPPRESS)
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a per-rank value over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def source_hash(kernel):
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "retrieval_block_sparse_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_lookup(kernel, workload, path=None):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    p = path or os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = source_hash(kernel)
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel \
+                    and parts[1] == want and parts[2] == workload:
+                return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML while running."""
+
+    NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+             0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, torch_device: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml as nv
+            import torch
+            nv.nvmlInit()
+            pr = torch.cuda.get_device_properties(torch_device)
+            try:
+                bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+                self.h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = nv.nvmlDeviceGetHandleByIndex(torch_device)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: clocks reported as unavailable
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((time.time(), sm, rs, pw))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"unavailable": getattr(self, "err", "nvml")}
+        sel = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples[-3:]
+        reasons = set()
+        for _, _, rs, _ in sel:
+            for bit, name in self.NAMES.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([s[1] for s in sel])) if sel else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(sel),
+                "power_w_max": max((s[3] for s in sel), default=None), "source": "nvml"}
+
+
+# ---------------------------------------------------------------------------
+# workload bookkeeping (sizes only; no method arithmetic)
+
+
+def attended_counts(idx, T, bs, sink, window):
+    """Tokens attended per (b, kv head) for block selection idx [B][Hkv][k]."""
+    w0 = max(T - window, 0)
+    base = min(sink, w0) + (T - w0)
+    lo = np.maximum(idx.astype(np.int64) * bs, sink)
+    hi = np.minimum((idx.astype(np.int64) + 1) * bs, w0)
+    return base + np.clip(hi - lo, 0, None).sum(axis=-1)
+
+
+def step_bytes(w, nc, idx):
+    es = 2 if w.dtype == "bf16" else 4
+    rep_es = 4 if w.rep_mode == "mean" else es
+    rep = w.batch * w.n_kv_heads * nc * w.n_rep * w.head_dim * rep_es
+    gathered = int(attended_counts(idx, w.context, w.block_size, w.sink, w.window).sum()) \
+        * w.head_dim * es * 2
+    return rep, gathered
+
+
+def count_kernel_nodes(graph):
+    """Kernel nodes in a captured torch CUDA graph (None if not introspectable)."""
+    try:
+        from cuda.bindings import runtime as rt
+    except Exception:
+        try:
+            from cuda import cudart as rt
+        except Exception:
+            return None
+    try:
+        raw = graph.raw_cuda_graph()
+        err, _, n = rt.cudaGraphGetNodes(raw, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(raw, n)
+        kinds = 0
+        for node in nodes:
+            e, t = rt.cudaGraphNodeGetType(node)
+            if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kinds += 1
+        return kinds
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import retrieval_block_sparse_b200 as rba
+    from retrieval_block_sparse_b200 import synth
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    x = synth.decode_inputs(w)
+
+    def to_dev(a):
+        if w.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(
+                torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+
+    def new_store():
+        return rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                         head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
+                         dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep, device=dev)
+
+    master = new_store()
+    master.k.copy_(to_dev(x["K"]))
+    master.v.copy_(to_dev(x["V"]))
+    aux = None
+    if w.rep_mode == "topr_attn":
+        aux = to_dev(x["probe"])
+    elif w.rep_mode == "external":
+        aux = to_dev(x["landmarks"]).reshape(w.batch, w.n_kv_heads, w.n_blocks, 1, w.head_dim)
+    master.memorize(None, None, first_block=0, n_blocks=w.n_blocks, aux=aux)
+    q = to_dev(x["q"])
+    first, nc = master.candidates(w.context, w.sink, w.window)
+    idx0, _, _ = master.decode_step(q, w.top_k, w.context, w.sink, w.window)
+    master.check()
+    rep_b, gath_b = step_bytes(w, nc, idx0.cpu().numpy())
+    bytes_step = rep_b + gath_b
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = args.replicas or max(2, math.ceil(4 * l2 / bytes_step))
+    stores = [master] + [new_store() for _ in range(R - 1)]
+    for s in stores[1:]:
+        s.k.copy_(master.k)
+        s.v.copy_(master.v)
+        if master.rep is not None:
+            s.rep.copy_(master.rep)
+    ws = [s.decode_workspace(w.top_k, w.context, w.sink, w.window) for s in stores]
+    outs = [torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+            for _ in stores]
+    lses = [torch.empty((w.batch, w.n_q_heads), dtype=torch.float32, device=dev) for _ in stores]
+    idxs = [torch.empty((w.batch, w.n_kv_heads, w.top_k), dtype=torch.int32, device=dev)
+            for _ in stores]
+
+    def step(r):
+        stores[r].decode_step(q, w.top_k, w.context, w.sink, w.window, workspace=ws[r],
+                              out=outs[r], lse=lses[r], idx=idxs[r])
+
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for r in range(R):  # eager warm-up of every replica before capture
+            step(r)
+    torch.cuda.synchronize(dev)
+    g_all = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all, stream=stream):
+        for r in range(R):
+            step(r)
+    g_one = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(r)
+        g_one.append(g)
+    kern_per_step = None
+    n_nodes = count_kernel_nodes(g_one[0])
+    if n_nodes:
+        kern_per_step = n_nodes
+
+    def run_steps(n):
+        full, rem = divmod(n, R)
+        for _ in range(full):
+            g_all.replay()
+        for r in range(rem):
+            g_one[r].replay()
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.05)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream), torch.cuda.nvtx.range("bench_timed"):
+        ev0.record(stream)
+        run_steps(args.steps)
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    for s in stores:
+        s.check()
+    ms_max = reduce_max(ms, dev)
+    steps_per_s = world * args.steps / (ms_max / 1e3)
+
+    # dominant kernel alone: split-K attention over the selected blocks
+    aws = [s.attend_workspace(w.top_k, w.context, w.sink, w.window) for s in stores]
+
+    def att(r):
+        stores[r].attend(q, idxs[r], w.context, w.sink, w.window, out=outs[r], lse=lses[r],
+                         workspace=aws[r])
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            att(r)
+    g_att = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_att, stream=stream):
+        for r in range(R):
+            att(r)
+    reps_att = max(1, 2000 // R)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_att.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps_att):
+            g_att.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    att_us = e0.elapsed_time(e1) * 1e3 / (reps_att * R)
+    # score kernel alone (rep-key stream)
+    scs = [torch.empty((w.batch, w.n_kv_heads, nc), dtype=torch.float32, device=dev)
+           for _ in stores]
+    g_sc = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            stores[r].score(q, w.context, w.sink, w.window, out=scs[r])
+    with torch.cuda.graph(g_sc, stream=stream):
+        for r in range(R):
+            stores[r].score(q, w.context, w.sink, w.window, out=scs[r])
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_sc.replay()
+        e0.record(stream)
+        for _ in range(reps_att):
+            g_sc.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    score_us = e0.elapsed_time(e1) * 1e3 / (reps_att * R)
+
+    pk = peaks()
+    att_gbs = gath_b / (att_us * 1e-6) / 1e9
+    step_us = ms_max * 1e3 / args.steps
+    step_gbs = bytes_step / (step_us * 1e-6) / 1e9
+    traffic = traffic_lookup("attend_decode_kernel", args.workload)
+
+    # end to end through the host-buffer entry point
+    e2e = None
+    if args.e2e_steps > 0:
+        q_host = torch.empty_like(q, device="cpu").pin_memory()
+        q_host.copy_(q.cpu())
+        out_h = torch.empty(outs[0].shape, dtype=torch.float32).pin_memory()
+        lse_h = torch.empty(lses[0].shape, dtype=torch.float32).pin_memory()
+        idx_h = torch.empty(idxs[0].shape, dtype=torch.int32).pin_memory()
+        q_devs = [torch.empty_like(q) for _ in stores]
+
+        def e2e_step(i):
+            r = i % R
+            stores[r].decode_step_host(q_host, w.top_k, w.context, w.sink, w.window,
+                                       q_dev=q_devs[r], idx_dev=idxs[r], out_dev=outs[r],
+                                       lse_dev=lses[r], out_host=out_h, lse_host=lse_h,
+                                       idx_host=idx_h, workspace=ws[r])
+        with torch.cuda.stream(stream):
+            for i in range(min(20, args.e2e_steps)):
+                e2e_step(i)
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for i in range(args.e2e_steps):
+                e2e_step(i)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = reduce_max(e0.elapsed_time(e1), dev)
+        e2e = {"value": round(world * args.e2e_steps / (e_ms / 1e3), 2), "unit": UNIT,
+               "h2d_bytes_per_step": q.numel() * q.element_size(),
+               "d2h_bytes_per_step": out_h.numel() * 4 + lse_h.numel() * 4 + idx_h.numel() * 4,
+               "steps": args.e2e_steps, "call": "rba_decode_step_host (pinned host buffers)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, x, args.cpu_seconds, args.workload)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    launches = kern_per_step if kern_per_step else (3 if nc <= 8192 else 6)
+    line = {
+        "metric": METRIC, "value": round(steps_per_s, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_us / 1e3, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generator; K,V~N(0,1), planted per-head bias, 16-query probe)",
+        "config": {"workload": args.workload, "batch": w.batch, "q_heads": w.n_q_heads,
+                   "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context": w.context,
+                   "block_size": w.block_size, "rep_keys": w.n_rep, "top_k": w.top_k,
+                   "sink": w.sink, "window": w.window, "candidates": nc,
+                   "l2": f"inputs larger than L2: {R} store replicas rotated "
+                         f"({R} x {bytes_step / 1e6:.1f} MB >= 4 x {l2 / 1e6:.0f} MB L2)",
+                   "parallelism": f"replicas x{world} (no exchange step)"},
+        "roofline": {"bound": "hbm", "kernel": "attend_decode_kernel",
+                     "achieved": round(att_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(att_gbs / pk["hbm_gbs"], 4),
+                     "peak_source": f"{pk['source']} (MEASURED_PEAKS.json hbm_gbs)"
+                     if pk["source"] == "measured" else "fallback 6650 GB/s",
+                     "traffic": traffic, "algorithmic_bytes": gath_b,
+                     "launch_us": round(att_us, 3)},
+        "step": {"algorithmic_bytes": bytes_step, "rep_key_bytes": rep_b,
+                 "gathered_kv_bytes": gath_b, "us": round(step_us, 3),
+                 "achieved_gbs": round(step_gbs, 1),
+                 "frac_of_hbm": round(step_gbs / pk["hbm_gbs"], 4),
+                 "score_kernel_us": round(score_us, 3),
+                 "score_kernel_gbs": round(rep_b / (score_us * 1e-6) / 1e9, 1)},
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": launches * args.steps,
+        "kernels_per_step": launches,
+        "cpu_baseline": cpu,
+    }
+    return line
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline / reference arm: the fp64 oracle, as it stands
+
+
+def _blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def _oracle_units(w, x):
+    """One (batch, kv head) unit of the decode step, as the oracle computes it."""
+    import oracle as O
+    probe = O.widen(x["probe"], w.dtype) if "probe" in x else None
+    reps = None
+    if w.rep_mode != "identity":
+        reps = np.zeros((w.batch, w.n_kv_heads, w.n_blocks, w.n_rep, w.head_dim))
+        for b in range(w.batch):
+            for h in range(w.n_kv_heads):
+                if w.rep_mode == "external":
+                    reps[b, h, :, 0] = O.widen(x["landmarks"][b, h], w.dtype)
+                    continue
+                K = O.widen(x["K"][b, h, :w.n_blocks * w.block_size], w.dtype)
+                reps[b, h] = O.memorize(K, w.rep_mode, w.block_size, w.n_rep,
+                                        probe=None if probe is None else probe[h])[0]
+    g = w.n_q_heads // w.n_kv_heads
+    units = [(b, h) for b in range(w.batch) for h in range(w.n_kv_heads)]
+
+    def unit(i):
+        b, h = units[i % len(units)]
+        O.decode(x["q"][b:b + 1, h * g:(h + 1) * g], x["K"][b:b + 1, h:h + 1],
+                 x["V"][b:b + 1, h:h + 1], None if reps is None else reps[b:b + 1, h:h + 1],
+                 dtype=w.dtype,
+                 block_size=w.block_size, sink=w.sink, window=w.window, top_k_blocks=w.top_k)
+    return unit, len(units)
+
+
+def cpu_baseline(w, x, seconds, workload=WORKLOAD):
+    unit, per_step = _oracle_units(w, x)
+    unit(0)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        unit(n)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and n >= per_step:
+            break
+    return {"value": round(n / el / per_step, 4), "unit": UNIT, "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} (batch, kv head) units = {n / per_step:.2f} decode steps of {workload} "
+                      f"(score + top-k + attend, fp64 numpy; memorise excluded), {el:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    from retrieval_block_sparse_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    x = synth.decode_inputs(w)
+    unit, per_step = _oracle_units(w, x)
+    for i in range(min(args.warmup, per_step)):
+        unit(i)
+    # each reference step is one (batch, kv head) unit; capped at 240 s of work
+    t0 = time.perf_counter()
+    n = 0
+    while n < args.steps:
+        unit(n)
+        n += 1
+        if time.perf_counter() - t0 > 240.0:
+            break
+    el = time.perf_counter() - t0
+    value = n / el / per_step
+    sample = (f"{n} (batch, kv head) units of {args.workload} (each 1/{per_step} of a decode step: "
+              f"score + top-k + attend, fp64 numpy)" +
+              (f"; stopped at the 240 s cap before {args.steps}" if n < args.steps else ""))
+    cores = _blas_threads()
+    return {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": n, "warmup": args.warmup, "ms_per_step": round(el * 1e3 / n * per_step, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded generator)", "impl": "reference",
+            "config": {"workload": args.workload},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse(argv)
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

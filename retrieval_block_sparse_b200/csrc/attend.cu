@@ -63,8 +63,7 @@ rba_status launch_t(const AttendArgs& a, int BH, cudaStream_t stream) {
                       size_t(2 * a.k + 5) * 4 + size_t(G) * a.nsplit * 4 + 16;
   if (smem > 227 * 1024) return RBA_ERR_UNSUPPORTED;
   auto kfn = attend_decode_kernel<T, D, G>;
-  RBA_CUDA_TRY(cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(smem)));
+  RBA_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kfn), smem));
   kfn<<<dim3(a.nsplit, BH), kAttendThreads, smem, stream>>>(a);
   RBA_LAUNCH_CHECK();
   return RBA_OK;
@@ -221,7 +220,7 @@ rba_status rba_decode_step(const rba_store* st, const void* q, int32_t k, int64_
                            int32_t* idx, float* out, float* lse, void* workspace,
                            size_t ws_bytes, cudaStream_t stream) {
   using namespace rba;
-  if (st == nullptr || q == nullptr || out == nullptr || idx == nullptr || k < 0)
+  if (st == nullptr || q == nullptr || out == nullptr || k < 0 || (k > 0 && idx == nullptr))
     return RBA_ERR_INVALID_ARG;
   if (st->d.mode == RBA_REP_EMBED_COSINE) return RBA_ERR_INVALID_ARG;
   Geometry g;

@@ -239,9 +239,7 @@ extern "C" rba_status rba_memorize(rba_store* st, const void* k_src, const void*
 #define RBA_TOPR(T_, D_)                                                                      \
   do {                                                                                        \
     auto kfn = rep_topr_kernel<T_, D_>;                                                       \
-    if (smem > 48 * 1024)                                                                     \
-      RBA_CUDA_TRY(cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
-                                        static_cast<int>(smem)));                             \
+    RBA_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kfn), smem));                       \
     kfn<<<grid, threads, smem, stream>>>(static_cast<const T_*>(st->k),                       \
                                          static_cast<const T_*>(aux), static_cast<T_*>(st->rep), \
                                          st->rep_pos, d.n_kv_heads, static_cast<int>(bs),     \

@@ -124,6 +124,10 @@ struct Geometry {
 rba_status geometry(const rba_store* st, int64_t T, int32_t sink, int32_t window, Geometry* g);
 int num_sms();
 
+// Raises a kernel's dynamic shared-memory limit once per (device, kernel);
+// later calls (including inside stream capture) make no CUDA call.
+cudaError_t ensure_smem(const void* kernel, size_t bytes);
+
 #define RBA_CUDA_TRY(expr)                          \
   do {                                              \
     cudaError_t e_ = (expr);                        \

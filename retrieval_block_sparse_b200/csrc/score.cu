@@ -113,8 +113,7 @@ rba_status launch_score_cos(const rba_store* st, const float* qe, int n_q, const
   if (g.nc == 0 || n_q == 0) return RBA_OK;
   const size_t smem = size_t(d_ret) * sizeof(float);
   if (smem > 48 * 1024)
-    RBA_CUDA_TRY(cudaFuncSetAttribute(score_cos_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(smem)));
+    RBA_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(score_cos_kernel), smem));
   score_cos_kernel<<<n_q, 256, smem, stream>>>(qe, static_cast<const float*>(st->rep), scores,
                                                d_ret, g.first, g.nc);
   RBA_LAUNCH_CHECK();

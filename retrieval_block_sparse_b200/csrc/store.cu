@@ -1,5 +1,7 @@
 // Block store description, candidate geometry, status handling.
+#include <mutex>
 #include <new>
+#include <unordered_map>
 
 #include "rba_internal.cuh"
 
@@ -40,6 +42,23 @@ int num_sms() {
       cached = 148;
   }
   return cached;
+}
+
+cudaError_t ensure_smem(const void* kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static std::mutex mu;
+  static std::unordered_map<uint64_t, size_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t key = reinterpret_cast<uint64_t>(kernel) ^ (uint64_t(dev) << 56);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e == cudaSuccess) done[key] = bytes;
+  return e;
 }
 
 }  // namespace rba

@@ -89,9 +89,7 @@ rba_status launch_topk(const float* scores, int rows, int n, int k, int index_ba
     const int Pk = pow2_at_least(k < 2 ? 2 : k);
     const size_t smem = size_t(P) * 8 + size_t(Pk) * 4;
     if (smem > 48 * 1024)
-      RBA_CUDA_TRY(cudaFuncSetAttribute(topk_small_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(smem)));
+      RBA_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(topk_small_kernel), smem));
     topk_small_kernel<<<rows, kThreads, smem, stream>>>(scores, n, k, P, Pk, index_base, idx);
     RBA_LAUNCH_CHECK();
     return RBA_OK;

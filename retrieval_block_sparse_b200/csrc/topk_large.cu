@@ -273,8 +273,7 @@ rba_status launch_topk_large(const float* scores, int rows, int n, int k, int in
   int Pk = 2;
   while (Pk < k) Pk <<= 1;
   const size_t smem = size_t(kSortMax) * 8 + size_t(Pk) * 4;
-  RBA_CUDA_TRY(cudaFuncSetAttribute(finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(smem)));
+  RBA_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(finish_kernel), smem));
   finish_kernel<<<rows, kFinishThreads, smem, stream>>>(L.state, L.above, L.cand, n, k, Pk,
                                                         index_base, idx);
   RBA_LAUNCH_CHECK();
