@@ -180,6 +180,30 @@ rba_status rba_attend(const rba_store* store, const void* q, const int32_t* idx,
 size_t rba_attend_workspace_size(const rba_store* store, int32_t k, int64_t T, int32_t sink,
                                  int32_t window);
 
+/* rba_attend without a workspace argument, for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is an interface addition
+ * of this library.
+ * Meant for hosts that own all device memory through their own allocator (for
+ * example a serving engine that reserves HBM when it starts) and for call sites
+ * that cannot afford the device-wide synchronisation cudaMalloc may cause.
+ * Same computation, arguments, layouts and errors as rba_attend; the split
+ * partials and merge tickets live in a fixed device array inside the library,
+ * RBA_ATTEND_NOALLOC_SCRATCH_BYTES long, which every GPU that loads the library
+ * holds until the process exits.
+ *   - Allocates nothing: no cudaMalloc / cudaFree and no allocating library call.
+ *   - The first call on each device looks up the array's device address, with
+ *     that device current; make that first call before any stream capture.
+ *   - Each call zeroes the array's ticket region on `stream`, then launches.
+ *   - Every call shares the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other host threads) race and
+ *     must be serialised by the caller.
+ *   - A call needing more scratch than the limit (see rba_attend_workspace_size)
+ *     returns RBA_ERR_WORKSPACE and launches nothing. */
+#define RBA_ATTEND_NOALLOC_SCRATCH_BYTES ((size_t)2 << 20)
+rba_status rba_attend_noalloc(const rba_store* store, const void* q, const int32_t* idx,
+                              int32_t k, int64_t T, int32_t sink, int32_t window, float scale,
+                              float* out, float* lse, cudaStream_t stream);
+
 /* Chunked prefill, retrieval-causal ([ML] 2.3.3 / Figure 3): every row of a
  * query chunk attends bidirectionally to sink U retrieved blocks U window of
  * the memory, and causally to the chunk's own tokens (own token i' visible to

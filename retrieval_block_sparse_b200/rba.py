@@ -35,6 +35,8 @@ SIGNATURES = {
     "rba_attend": (_c_i32, [_p, _p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32, _p, _p, _p,
                             _c_size, _p]),
     "rba_attend_workspace_size": (_c_size, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
+    "rba_attend_noalloc": (_c_i32, [_p, _p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32, _p, _p,
+                                    _p]),
     "rba_attend_prefill": (_c_i32, [_p, _p, _c_i32, _c_i32, _p, _c_i32, _c_i32, _c_i64, _c_i32,
                                     _c_i32, _p, _p, _c_f32, _p, _p, _p, _c_size, _p]),
     "rba_attend_prefill_workspace_size": (_c_size, [_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i64,

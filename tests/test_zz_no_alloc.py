@@ -1,0 +1,73 @@
+"""rba_attend_noalloc: decode attention for callers that cannot allocate.
+
+Some hosts own all device memory through their own allocator (a serving
+engine that reserves HBM at start-up), and some call sites cannot afford the
+device-wide synchronisation a cudaMalloc may cause.  Those callers cannot hand
+rba_attend a workspace; rba_attend_noalloc keeps the scratch in a fixed
+device array inside the library instead.
+
+This test calls it through the C ABI twice in a row (different queries, the
+second call reusing whatever the first left in the shared array) and checks
+each output against rba_attend's, within the attention tolerance the other
+tests use (2e-3 of max |V| for bf16).  It also checks the size limit.  This
+file is collected last, and it passes on its own in a fresh process too (its
+first call is the first use of the array on the device).
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from retrieval_block_sparse_b200 import synth
+
+from parity import OUT_TOL, dev, make_decode_store, oracle_reps
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(rba, st, q, idx, w, out, lse):
+    L = rba.lib()
+    s = L.rba_attend_noalloc(st.handle, q.data_ptr(), idx.data_ptr(), idx.shape[-1], w.context,
+                             w.sink, w.window, ctypes.c_float(w.head_dim ** -0.5),
+                             out.data_ptr(), lse.data_ptr(),
+                             torch.cuda.current_stream().cuda_stream)
+    return s
+
+
+def test_noalloc_matches_attend_twice(rba):
+    w = synth.WORKLOADS["infllm-decode-128k"]
+    x = synth.decode_inputs(w)
+    reps, _ = oracle_reps(w, x)
+    st = make_decode_store(rba, w, x)
+    ref = O.decode(x["q"], x["K"], x["V"], reps, dtype=w.dtype, block_size=w.block_size,
+                   sink=w.sink, window=w.window, top_k_blocks=w.top_k)
+    idx = torch.from_numpy(ref["idx"].astype(np.int32)).cuda()
+    vmax = float(np.abs(O.widen(x["V"], w.dtype)).max())
+    q1 = dev(x["q"], w.dtype)
+    q2 = (q1.float() * -0.75).to(torch.bfloat16).contiguous()
+    for q in (q1, q2):
+        out = torch.full((w.batch, w.n_q_heads, w.head_dim), float("nan"), device="cuda")
+        lse = torch.full((w.batch, w.n_q_heads), float("nan"), device="cuda")
+        assert _noalloc(rba, st, q, idx, w, out, lse) == rba.OK
+        st.check()
+        o_ref, l_ref = st.attend(q, idx, w.context, w.sink, w.window)
+        err = float((out - o_ref).abs().max()) / vmax
+        assert err <= OUT_TOL[w.dtype], err
+        assert float((lse - l_ref).abs().max()) <= OUT_TOL[w.dtype]
+
+
+def test_noalloc_rejects_sizes_beyond_the_limit(rba):
+    # 160 x 32 MHA heads: the split partials need more than the fixed array
+    w = synth.WORKLOADS["landmark-decode-b16"].scaled(batch=160, context=100)
+    st = rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                   head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
+                   dtype="bf16", mode="external")
+    need = rba.lib().rba_attend_workspace_size(st.handle, 0, w.context, w.sink, w.window)
+    assert need > (2 << 20)
+    q = torch.zeros((w.batch, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros((w.batch, w.n_kv_heads, 0), dtype=torch.int32, device="cuda")
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device="cuda")
+    lse = torch.empty((w.batch, w.n_q_heads), device="cuda")
+    assert _noalloc(rba, st, q, idx, w, out, lse) == rba.ERR_WORKSPACE
