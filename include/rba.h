@@ -238,6 +238,16 @@ rba_status rba_decode_step(const rba_store* store, const void* q, int32_t k, int
 size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t T,
                                       int32_t sink, int32_t window);
 
+/* How rba_decode_step runs this problem (host only; queries the device, launches nothing):
+ *   1   one persistent launch: scores, selection and attention fused; candidates per
+ *       (b, kv head) <= 8192, k <= 1024, GQA group of 1, 2 or 4
+ *   0   three launches (rba_score, rba_topk, rba_attend): outside those limits
+ *  -2   within the limits but no CTA of the fused kernel fits on an SM (three launches)
+ *  -3   a CUDA error while asking (three launches)
+ *  -4   invalid arguments (as rba_decode_step would report) */
+int32_t rba_decode_step_plan(const rba_store* store, int32_t k, int64_t T, int32_t sink,
+                             int32_t window);
+
 /* rba_decode_step from and to host memory: copies q_host (host, dtype [B][Hq][D]) into
  * q_dev, runs the step, copies out/lse/idx back into the host buffers (any of lse_host,
  * idx_host may be NULL), then synchronises `stream`.  q_dev, idx_dev, out_dev, lse_dev are

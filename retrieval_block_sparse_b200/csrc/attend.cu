@@ -7,6 +7,7 @@
 // attended tokens and the last CTA of each (batch, kv head) merges the split
 // partials by log-sum-exp (no CTA ever waits for another).
 #include "attend_impl.cuh"
+#include "decode_fused.cuh"
 #include "score_impl.cuh"
 #include "topk_impl.cuh"
 
@@ -156,6 +157,8 @@ rba_status launch_attend(const rba_store* st, const void* q, const int32_t* idx,
 namespace {
 
 struct StepWs {
+  void* fused_sync;
+  float* fused_slots;
   float* scores;
   void* topk_ws;
   size_t topk_bytes;
@@ -164,13 +167,17 @@ struct StepWs {
   size_t total;
 };
 
+// [fused sync words (zero)] [attend: tickets (zero) + partials] [scores]
+// [top-k scratch] [fused partial slots]: the zero words of the two paths
+// never overlap the other path's scratch.
 StepWs step_layout(void* ws, const rba_store* st, const Geometry& g, int k, bool own_scores) {
   const rba_store_desc& d = st->d;
   const int BH = d.batch * d.n_kv_heads;
   StepWs s;
   char* p = static_cast<char*>(ws);
   size_t off = 0;
-  // the attend workspace (with its zero tickets) comes first
+  s.fused_sync = p + off;
+  off += fused_sync_bytes(st);
   const int nsplit = attend_nsplit(BH, n_att_bound(g, k));
   s.attend_bytes = attend_workspace_bytes(BH, d.batch * d.n_q_heads, d.head_dim, nsplit);
   s.attend_ws = p + off;
@@ -183,6 +190,8 @@ StepWs step_layout(void* ws, const rba_store* st, const Geometry& g, int k, bool
   s.topk_bytes = topk_workspace(BH, g.nc, k);
   s.topk_ws = p + off;
   off += align_up(s.topk_bytes, 256);
+  s.fused_slots = reinterpret_cast<float*>(p + off);
+  off += fused_slot_bytes(st, g, k, nullptr);
   s.total = off;
   return s;
 }
@@ -233,6 +242,10 @@ rba_status rba_decode_step(const rba_store* st, const void* q, int32_t k, int64_
   const int BH = st->d.batch * st->d.n_kv_heads;
   const int grp = st->d.n_q_heads / st->d.n_kv_heads;
   if (grp > 64) return RBA_ERR_UNSUPPORTED;
+  if (fused_eligible(st, g, k)) {
+    s = launch_fused(st, q, k, g, scale, sc, idx, out, lse, w.fused_sync, w.fused_slots, stream);
+    if (s != RBA_ERR_UNSUPPORTED) return s;
+  }
   if (k > 0) {
     s = launch_score_dot(st, q, 1, nullptr, g, sc, stream);
     if (s != RBA_OK) return s;
@@ -240,6 +253,19 @@ rba_status rba_decode_step(const rba_store* st, const void* q, int32_t k, int64_
     if (s != RBA_OK) return s;
   }
   return launch_attend(st, q, idx, k, g, scale, out, lse, w.attend_ws, w.attend_bytes, stream);
+}
+
+int32_t rba_decode_step_plan(const rba_store* st, int32_t k, int64_t T, int32_t sink,
+                             int32_t window) {
+  using namespace rba;
+  Geometry g;
+  if (st == nullptr || k < 0 || geometry(st, T, sink, window, &g) != RBA_OK || k > g.nc)
+    return -4;
+  if (!fused_eligible(st, g, k)) return 0;
+  const int occ = fused_occupancy(st);
+  if (occ < 0) return -3;
+  if (occ == 0) return -2;
+  return 1;
 }
 
 size_t rba_decode_step_workspace_size(const rba_store* st, int32_t k, int64_t T, int32_t sink,

@@ -63,8 +63,15 @@ __global__ void hist_kernel(const float* __restrict__ scores, int n, uint32_t* _
   const float* s = scores + row * n;
   const int i0 = blockIdx.x * kChunk;
   const int i1 = min(n, i0 + kChunk);
-  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x)
-    atomicAdd(&h[ordered_f32(s[i]) >> kShift], 1u);
+  // lanes falling into the same bin add once (neighbouring scores share their
+  // top bits, so plain per-lane atomics would serialise)
+  for (int base = i0; base < i1; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const bool ok = i < i1;
+    const uint32_t bin = ok ? ordered_f32(s[i]) >> kShift : uint32_t(kBins);
+    const unsigned same = __match_any_sync(0xffffffffu, bin);
+    if (ok && (threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&h[bin], uint32_t(__popc(same)));
+  }
   __syncthreads();
   for (int b = threadIdx.x; b < kBins; b += blockDim.x)
     if (h[b]) atomicAdd(&hist[row * kBins + b], h[b]);

@@ -44,6 +44,7 @@ SIGNATURES = {
     "rba_decode_step": (_c_i32, [_p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32, _p, _p, _p, _p,
                                  _p, _c_size, _p]),
     "rba_decode_step_workspace_size": (_c_size, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
+    "rba_decode_step_plan": (_c_i32, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
     "rba_decode_step_host": (_c_i32, [_p, _p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32, _p, _p,
                                       _p, _p, _p, _p, _p, _c_size, _p]),
     "rba_store_check": (_c_i32, [_p, _p]),
@@ -253,6 +254,10 @@ class Store:
     def decode_workspace(self, k, T, sink, window):
         n = lib().rba_decode_step_workspace_size(self.handle, k, T, sink, window)
         return torch.zeros(max(n, 16), dtype=torch.uint8, device=self.k.device)
+
+    def decode_plan(self, k, T, sink, window):
+        """1: fused single launch; 0: three launches; <0: fused refused (see rba.h)."""
+        return lib().rba_decode_step_plan(self.handle, k, T, sink, window)
 
     def decode_step(self, q, k, T, sink, window, *, scale=None, workspace=None, out=None,
                     lse=None, idx=None, scores=None):

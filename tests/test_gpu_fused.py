@@ -1,0 +1,54 @@
+"""The whole decode step in one launch (rba_decode_step) against the
+three-launch path (rba_score -> rba_topk -> rba_attend) on the same store:
+identical selections, outputs within the attention tolerance.  Shapes cover
+one CTA per SM, grids smaller than the SM count, several heads per CTA, GQA
+groups of 1, 2 and 4, ragged block sizes, and repeated calls on one
+workspace (its synchronisation words must come back to zero)."""
+import numpy as np
+import pytest
+import torch
+
+from retrieval_block_sparse_b200 import synth
+
+from parity import OUT_TOL, dev, make_decode_store
+
+pytestmark = pytest.mark.gpu
+W = synth.WORKLOADS
+CASES = {
+    "infllm-decode-128k": W["infllm-decode-128k"],
+    "infllm-2k-window": W["infllm-decode-128k"].scaled(context=32768, window=2048, top_k=64),
+    "landmark-decode-b16": W["landmark-decode-b16"],
+    "tiny-decode-f32": W["tiny-decode-f32"],
+    "gqa2-bs24-f32": W["tiny-decode-f32"].scaled(n_q_heads=8, n_kv_heads=4, context=1000,
+                                                 block_size=24, sink=30, window=70, top_k=7),
+    "one-head": W["infllm-decode-128k"].scaled(n_q_heads=4, n_kv_heads=1, context=16384,
+                                               window=512, top_k=8),
+    "batch4-d64": W["landmark-decode-b16"].scaled(batch=4, n_q_heads=8, n_kv_heads=8,
+                                                  head_dim=64, context=3000, top_k=6),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fused_step_equals_three_launches(rba, name):
+    w = CASES[name]
+    x = synth.decode_inputs(w)
+    st = make_decode_store(rba, w, x)
+    q = dev(x["q"], w.dtype)
+    first, nc = st.candidates(w.context, w.sink, w.window)
+    scores = st.score(q, w.context, w.sink, w.window)
+    idx3 = rba.topk(scores.reshape(-1, nc), w.top_k, index_base=first).reshape(
+        w.batch, w.n_kv_heads, w.top_k)
+    out3, lse3 = st.attend(q, idx3, w.context, w.sink, w.window)
+    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 1
+    ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)
+    vmax = float(st.v.float().abs().max())
+    for rep in range(3):
+        sc = torch.empty_like(scores)
+        idx, out, lse = st.decode_step(q, w.top_k, w.context, w.sink, w.window, workspace=ws,
+                                       scores=sc)
+        st.check()
+        assert torch.equal(idx, idx3), rep
+        assert torch.allclose(sc, scores, rtol=1e-5, atol=1e-5)
+        err = float((out - out3).abs().max()) / vmax
+        assert err <= OUT_TOL[w.dtype], (rep, err)
+        assert float((lse - lse3).abs().max()) <= OUT_TOL[w.dtype]
