@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1) attend_decode_kernel(Attend
     cp_async_wait<C::NS - 1>();
     __syncthreads();
     consume_tile<T, D, G>(stages + (t % C::NS) * C::STAGE, min(C::TT, v_hi - v_lo - t * C::TT),
-                          st);
+                          st, threadIdx.x >> 5);
     __syncthreads();
   }
   write_partial<T, D, G>(a, bh, split, st, red);

@@ -34,22 +34,24 @@ struct AttendArgs {
 constexpr int kAttendWarps = 8;
 constexpr int kAttendThreads = kAttendWarps * 32;
 
-template <typename T, int D>
+// Tile geometry for NW consuming warps: each warp takes TPW rows per step,
+// NT steps per tile, LPR lanes per row and EPL elements per lane.
+template <typename T, int D, int NW = kAttendWarps>
 struct DecodeTile {
   static constexpr int ES = sizeof(T);
   static constexpr int EPL = 16;                  // elements of a row per lane
   static constexpr int LPR = D / EPL;             // lanes per row
   static constexpr int TPW = 32 / LPR;            // rows per warp step
   static constexpr int NT = 2;                    // steps per tile
-  static constexpr int TT = kAttendWarps * TPW * NT;  // tokens per tile
+  static constexpr int TT = NW * TPW * NT;        // tokens per tile
   static constexpr int ROWB = D * ES;
   static constexpr int CPR = ROWB / 16;           // 16-byte chunks per row
   static constexpr int CPL = EPL * ES / 16;       // chunks per lane per row
   static constexpr int EPC = 16 / ES;             // elements per chunk
-  static constexpr int NS = ES == 2 ? 3 : 2;      // pipeline stages
+  static constexpr int NS = ES == 2 ? 3 : 2;      // pipeline stages (split-K kernel)
   static constexpr int STAGE = 2 * TT * ROWB;     // K tile + V tile
-  static constexpr int LOADS = 2 * TT * CPR / kAttendThreads;  // cp.async per thread per tile
-  static_assert((2 * TT * CPR) % kAttendThreads == 0, "tile must split over the CTA");
+  static constexpr int LOADS = 2 * TT * CPR / (NW * 32);  // cp.async per thread per tile
+  static_assert((2 * TT * CPR) % (NW * 32) == 0, "tile must split over the warps");
 };
 
 // ---------------------------------------------------------------------------
@@ -216,12 +218,13 @@ __device__ __forceinline__ void load_slice(const char* row, int part, int rot, f
   }
 }
 
-// Consume one staged tile of `nvalid` rows.
-template <typename T, int D, int G>
+// Consume one staged tile of `nvalid` rows; `warp` is this warp's index
+// among the NW consuming warps (it owns rows [warp * TPW * NT, +TPW * NT)).
+template <typename T, int D, int G, int NW = kAttendWarps>
 __device__ __forceinline__ void consume_tile(const char* stage, int nvalid,
-                                             LaneState<T, D, G>& st) {
-  using C = DecodeTile<T, D>;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+                                             LaneState<T, D, G>& st, int warp) {
+  using C = DecodeTile<T, D, NW>;
+  const int lane = threadIdx.x & 31;
   const int slot = lane / C::LPR, part = lane % C::LPR;
   const int rot = lane_rot<T, D>(part);
   const char* sK = stage;

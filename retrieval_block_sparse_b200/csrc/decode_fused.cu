@@ -5,22 +5,24 @@
 // "method" and "overall framework"; Landmark Attention review, "proposed
 // method"; MemLong summary, 2.3.2 TopK and 2.3.3).  What this launch adds is
 // the schedule:
-//   * one CTA per SM, 8 warps;
-//   * every CTA gets an equal share of three flattened work lists, processed
-//     in order: (1) candidate blocks to score, (2) sink + window rows, which
-//     need no selection, (3) rows of the selected blocks;
-//   * warp 0 stages each item ahead of use with bulk asynchronous copies
-//     (whole contiguous runs: rep keys of consecutive candidates, K/V rows of
-//     a segment) into a ring of shared-memory stages guarded by mbarriers;
-//   * the last CTA to finish scoring a (batch, kv head) runs its top-k and
-//     publishes a ready flag; a CTA waits for that flag (bounded) only when
-//     it stages that head's selected blocks, and only after publishing its
-//     own selections, so selection overlaps the sink/window stream and no
-//     wait can be circular;
-//   * partial softmax states go to per-(head, phase, CTA) slots; the last
+//   * one CTA per SM: warp 0 only stages data, warps 1..7 compute;
+//   * every CTA gets an equal share of two flattened work lists, processed
+//     in order: (1) candidate blocks to score, (2) attention rows, where each
+//     head's share mixes sink + window rows (no selection needed) and rows of
+//     the selected blocks in proportion;
+//   * warp 0 walks the same item sequence as the compute warps and stages
+//     each item with bulk asynchronous copies (whole contiguous runs: rep keys
+//     of consecutive candidates, K/V rows of a segment) into a ring of
+//     shared-memory stages guarded by full / empty mbarriers, waiting for a
+//     head's selection only when it reaches that head's selected rows;
+//   * the last CTA to finish scoring a (batch, kv head) selects its top-k and
+//     publishes a ready flag; selection overlaps the sink/window stream;
+//   * partial softmax states go to per-(head, CTA) slots; the last
 //     contributor of a head merges them (no CTA waits for a merge).
-// All cross-CTA waits are bounded in time; on expiry the kernel records
-// RBA_ERR_TIMEOUT in the status word, skips the work, and still terminates.
+// No wait can be circular: scoring depends only on a CTA's own stager, and
+// every CTA scores before it attends.  All waits are bounded in time; on
+// expiry the kernel records RBA_ERR_TIMEOUT in the status word, skips the
+// remaining work, waits (bounded) for its copies in flight and terminates.
 #include <cstdio>
 #include <cstdlib>
 
@@ -30,18 +32,19 @@
 namespace rba {
 namespace {
 
-constexpr int kCW = 8;                        // compute warps
+constexpr int kCW = 7;                        // compute warps (warps 1..7)
 constexpr int kCT = kCW * 32;                 // compute threads
-constexpr int kFT = kCT;                      // warp 0 also stages the items
+constexpr int kFT = kCT + 32;                 // + warp 0, which stages
 constexpr int kMaxN = 8192;                   // candidates per (b, kv head)
 constexpr int kMaxK = 1024;
 constexpr int kMaxTouch = 64;                 // heads one CTA's score range may touch
-constexpr int kMaxStages = 4;
-constexpr int kMaxSlots = 128;                // partial slots per head (both phases)
+constexpr int kMaxStages = 6;
+constexpr int kMaxSlots = 128;                // partial slots per head
 constexpr int kMinRowsPerCta = 128;           // grid shrinks for small problems
 constexpr int kMaxGrid = 256;                 // CTAs (one per SM)
+constexpr int kBins = 256;                    // value bins of the top-k select
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
-static_assert(kCW == kAttendWarps, "tile geometry assumes the decode-attention warp count");
+static_assert(kMaxTouch * 128 <= kMaxN, "summed queries share the top-k key buffer");
 
 struct FusedArgs {
   AttendArgs at;            // K, V, q, out, lse, status, cap, T, w0, Hq, Hkv, k, bs, sink,
@@ -94,14 +97,33 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// bounded wait on an mbarrier phase; false on timeout
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
-  if (mbar_try(b, parity)) return true;
+// Warp-uniform bounded wait on an mbarrier phase (every lane acquires it).
+// False when the CTA is aborting or the wait ran out (then reported, and
+// the abort flag set).
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status, int where) {
+  bool ok = mbar_try(b, parity);
+  if (__all_sync(0xffffffffu, ok)) return true;
   const unsigned long long t0 = now_ns();
-  while (!mbar_try(b, parity)) {
-    if (now_ns() - t0 > kTimeoutNs) return false;
+  while (true) {
+    if (!ok) ok = mbar_try(b, parity);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
+    if (__shfl_sync(0xffffffffu, now_ns() - t0 > kTimeoutNs, 0)) {
+      if ((threadIdx.x & 31) == 0) {
+        report(status, RBA_ERR_TIMEOUT, kWhereFused, where);
+        *abort_flag = 1;
+      }
+      __syncwarp();
+      return false;
+    }
   }
-  return true;
+}
+// bounded wait that ignores the abort flag (draining copies in flight)
+__device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
+  const unsigned long long t0 = now_ns();
+  while (!mbar_try(b, parity) && now_ns() - t0 <= kTimeoutNs) {
+  }
 }
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
                                          uint64_t* bar) {
@@ -119,9 +141,20 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
 __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+// barrier of the compute warps only (warp 0 never joins it)
 __device__ __forceinline__ void compute_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
 }
+__device__ __forceinline__ int ctid() { return static_cast<int>(threadIdx.x) - 32; }
+__device__ __forceinline__ int cwarp() { return static_cast<int>(threadIdx.x >> 5) - 1; }
 
 // ---------------------------------------------------------------------------
 // work lists
@@ -189,9 +222,8 @@ __device__ __forceinline__ void attn_head(const FusedArgs& a, Iter& it) {
   it.sel1 = static_cast<int>(x1 - s1);
 }
 
-// B0 / B1: CTA boundaries bnd(0..P) of the candidate and attention lists
-__device__ __forceinline__ void iter_begin(const FusedArgs& a, Iter& it, const int64_t* B0,
-                                           const int64_t* B1) {
+// B0: CTA boundaries bnd(0..P) of the candidate list
+__device__ __forceinline__ void iter_begin(const FusedArgs& a, Iter& it, const int64_t* B0) {
   it.phase = 0;
   it.r = B0[blockIdx.x];
   it.r1 = B0[blockIdx.x + 1];
@@ -199,9 +231,9 @@ __device__ __forceinline__ void iter_begin(const FusedArgs& a, Iter& it, const i
     it.bh = static_cast<int>(it.r / a.at.nc);
     it.loc = static_cast<int>(it.r - int64_t(it.bh) * a.at.nc);
   }
-  (void)B1;
 }
 
+// B1: CTA boundaries of the attention list
 template <int TT>
 __device__ __forceinline__ bool next_item(const FusedArgs& a, Iter& it, Item& out,
                                           const int64_t* B1) {
@@ -268,45 +300,38 @@ struct __align__(16) Meta {
 
 template <typename T, int D, int G>
 struct FusedSmem {
-  using C = DecodeTile<T, D>;
+  using C = DecodeTile<T, D, kCW>;
   static constexpr int STAGE = C::STAGE;
   // regions after the stage ring (NS * STAGE, chosen at launch)
-  static constexpr int RED = kCW * G * (D + 2) * 4;             // warp states / merge sums
+  static constexpr int up16(int x) { return (x + 15) & ~15; }
+  static constexpr int RED = up16(kCW * G * (D + 2) * 4);       // warp states / merge sums
   static constexpr int SEL = (kMaxK + 4) * 4 * 2;               // selected prefix + starts
-  static constexpr int SLOTS = (kMaxSlots + 3 * G * kMaxSlots) * 4;  // merge: list, m, l, w
+  static constexpr int SLOTS = up16((kMaxSlots + 3 * G * kMaxSlots) * 4);  // merge: m, l, w
   static constexpr int MISC = 4096;
-  static constexpr int KEYS = kMaxN * 4;                        // top-k keys of one head
+  static constexpr int KEYS = kMaxN * 4;      // top-k values or keys; summed queries first
+  static constexpr int FLAGS = kMaxN + kCT * 4;  // top-k: selected flags, boundary-bin members
   static constexpr int BOUNDS = 2 * (kMaxGrid + 1) * 8;         // CTA boundaries, 2 lists
   static size_t bytes(int NS) {
-    return size_t(NS) * STAGE + RED + SEL + SLOTS + MISC + KEYS + BOUNDS;
+    return size_t(NS) * STAGE + RED + SEL + SLOTS + MISC + KEYS + FLAGS + BOUNDS;
   }
 };
 
 // ---------------------------------------------------------------------------
-// block-wide helpers
-
-__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "l"(p), "r"(v)
-               : "memory");
-  return old;
-}
+// compute-warp helpers
 
 __device__ __forceinline__ int compute_exclusive_scan(int v, int* s_w, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, cw = cwarp();
   int incl = v;
   for (int o = 1; o < 32; o <<= 1) {
     const int t = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += t;
   }
-  if (lane == 31) s_w[warp] = incl;
+  if (lane == 31) s_w[cw] = incl;
   compute_sync();
   int base = 0, tot = 0;
   for (int w = 0; w < kCW; ++w) {
     const int x = s_w[w];
-    if (w < warp) base += x;
+    if (w < cw) base += x;
     tot += x;
   }
   compute_sync();
@@ -314,16 +339,28 @@ __device__ __forceinline__ int compute_exclusive_scan(int v, int* s_w, int* tota
   return base + incl - v;
 }
 
-// Exact top-k of row bh (n <= kMaxN scores in global memory) by the CTA:
-// radix select of the k-th largest order-preserving score value, then ties
-// at that value taken in position order; positions written ascending.
-__device__ __forceinline__ void topk_row(const FusedArgs& a, int bh, uint32_t* hist, int* s_w,
-                                         int* s_misc, uint32_t* keys) {
+// Positions whose flag is set, written ascending to idx[bh] (first + j).
+__device__ __forceinline__ void write_selected(const FusedArgs& a, int bh, const uint8_t* flag,
+                                               int* s_w) {
+  const int n = a.at.nc;
+  const int per = (n + kCT - 1) / kCT;
+  const int p0 = ctid() * per, p1 = min(n, p0 + per);
+  int cnt = 0;
+  for (int j = p0; j < p1; ++j) cnt += flag[j];
+  int tot;
+  int rank = compute_exclusive_scan(cnt, s_w, &tot);
+  int32_t* dst = a.idx + int64_t(bh) * a.at.k;
+  for (int j = p0; j < p1; ++j)
+    if (flag[j]) dst[rank++] = a.at.first + j;
+}
+
+// Exact top-k of row bh by the radix select of the k-th largest
+// order-preserving score value; ties at that value go to the lower
+// positions.  `keys` holds kMaxN words.
+__device__ __noinline__ void topk_radix(const FusedArgs& a, int bh, uint32_t* hist, int* s_w,
+                                        int* s_misc, uint32_t* keys, uint8_t* flag) {
   const int n = a.at.nc, k = a.at.k;
-  const int tid = threadIdx.x;
-  const int per = (n + kCT - 1) / kCT;  // positions [p0, p0 + per) belong to this thread
-  const int p0 = tid * per;
-  const int p1 = min(n, p0 + per);
+  const int tid = ctid(), lane = threadIdx.x & 31;
   const float* s = a.scores + int64_t(bh) * n;
   for (int j = tid; j < n; j += kCT) keys[j] = ordered_f32(__ldcg(s + j));
   compute_sync();
@@ -332,15 +369,14 @@ __device__ __forceinline__ void topk_row(const FusedArgs& a, int bh, uint32_t* h
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int b = tid; b < 256; b += kCT) hist[b] = 0;
     compute_sync();
-    // lanes falling into the same bin add once (scores of one head share
-    // their top bits, so plain per-lane atomics would serialise)
-    for (int j0 = tid - (tid & 31); j0 < n; j0 += kCT) {
-      const int j = j0 + (tid & 31);
+    // lanes falling into the same bin add once
+    for (int j0 = tid - lane; j0 < n; j0 += kCT) {
+      const int j = j0 + lane;
       const uint32_t u = j < n ? keys[j] : 0u;
       const bool in = j < n && (u & mask) == prefix;
       const uint32_t bin = in ? ((u >> shift) & 255u) : 256u;
       const unsigned same = __match_any_sync(0xffffffffu, bin);
-      if (in && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], uint32_t(__popc(same)));
+      if (in && lane == __ffs(same) - 1) atomicAdd(&hist[bin], uint32_t(__popc(same)));
     }
     compute_sync();
     if (tid < 32) {
@@ -372,34 +408,160 @@ __device__ __forceinline__ void topk_row(const FusedArgs& a, int bh, uint32_t* h
     kk -= s_misc[1];
     compute_sync();
   }
-  // prefix = the k-th largest value: take every larger score and the first
-  // kk equal ones in position order; write positions in ascending order
+  // prefix = the k-th largest value: every larger score, and the first kk
+  // equal ones in position order
+  const int per = (n + kCT - 1) / kCT;
+  const int p0 = tid * per, p1 = min(n, p0 + per);
   int n_eq = 0;
   for (int j = p0; j < p1; ++j) n_eq += keys[j] == prefix;
   int tot;
-  int eq_rank = compute_exclusive_scan(n_eq, s_w, &tot);
-  int n_sel = 0;
-  for (int j = p0, e = eq_rank; j < p1; ++j) {
+  int e = compute_exclusive_scan(n_eq, s_w, &tot);
+  for (int j = p0; j < p1; ++j) {
     const uint32_t u = keys[j];
-    n_sel += u > prefix || (u == prefix && e++ < kk);
+    flag[j] = u > prefix || (u == prefix && e++ < kk);
   }
-  int rank = compute_exclusive_scan(n_sel, s_w, &tot);
-  int32_t* dst = a.idx + int64_t(bh) * k;
-  for (int j = p0, e = eq_rank; j < p1; ++j) {
-    const uint32_t u = keys[j];
-    if (u > prefix || (u == prefix && e++ < kk)) dst[rank++] = a.at.first + j;
-  }
+  compute_sync();
+  write_selected(a, bh, flag, s_w);
   compute_sync();
 }
 
-// Stages one item into `stg` (warp 0, all lanes): bulk copies that complete
-// on `bar`, whose transaction count is armed with the item's bytes.
-// Returns 1 staged, 0 not staged yet (selection not published and may_wait
-// is false; nothing armed), -1 timed out (stage armed empty).
+// value bin of x: monotone non-decreasing in x, so every score in a higher
+// bin is strictly larger than every score in a lower one
+__device__ __forceinline__ int value_bin(float x, float lo, float scale) {
+  const float t = __fmul_rn(__fsub_rn(x, lo), scale);
+  return min(kBins - 1, static_cast<int>(t));
+}
+
+// Exact top-k of row bh (1 <= k < n) with one histogram pass: kBins bins
+// linear in the score value between the row's min and max; every score in
+// the bins above the bin holding the k-th largest is selected, and inside
+// that bin the members are ranked exactly (value, then lower position).
+// Returns false (nothing written) for rows it does not cover -- non-finite
+// scores, a zero range, or more members in the boundary bin than compute
+// threads -- which the radix select then takes.
+__device__ __noinline__ bool topk_binned(const FusedArgs& a, int bh, uint32_t* hist, int* s_w,
+                                         int* s_misc, float* s_f, float* vals, uint8_t* flag,
+                                         int* cand) {
+  const int n = a.at.nc, k = a.at.k;
+  const int tid = ctid(), lane = threadIdx.x & 31, cw = cwarp();
+  const float* s = a.scores + int64_t(bh) * n;
+  float lo = INFINITY, hi = -INFINITY;
+  int bad = 0;
+  for (int j = tid; j < n; j += kCT) {
+    const float v = __ldcg(s + j);
+    vals[j] = v;
+    bad |= !isfinite(v);
+    lo = fminf(lo, v);
+    hi = fmaxf(hi, v);
+  }
+  for (int b = tid; b < kBins; b += kCT) hist[b] = 0;
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    s_f[2 * cw] = lo;
+    s_f[2 * cw + 1] = hi;
+    s_w[cw] = bad;
+  }
+  compute_sync();
+  lo = s_f[0];
+  hi = s_f[1];
+  bad = s_w[0];
+  for (int w = 1; w < kCW; ++w) {
+    lo = fminf(lo, s_f[2 * w]);
+    hi = fmaxf(hi, s_f[2 * w + 1]);
+    bad |= s_w[w];
+  }
+  const float range = hi - lo;
+  const float scale = float(kBins) / range;
+  // (uniform: every compute thread decides on the same shared values)
+  if (bad || !(range > 0.f) || !isfinite(range) || !isfinite(scale)) return false;
+  for (int j0 = tid - lane; j0 < n; j0 += kCT) {
+    const int j = j0 + lane;
+    const int bin = j < n ? value_bin(vals[j], lo, scale) : kBins;
+    const unsigned same = __match_any_sync(0xffffffffu, bin);
+    if (j < n && lane == __ffs(same) - 1) atomicAdd(&hist[bin], uint32_t(__popc(same)));
+  }
+  compute_sync();
+  if (cw == 0) {
+    // lane l owns bins [8l, 8l+8); counts above a bin = all higher bins
+    uint32_t c[8], tot = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      c[i] = hist[lane * 8 + i];
+      tot += c[i];
+    }
+    uint32_t incl = tot;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += t;
+    }
+    uint32_t above = incl - tot;
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+      if (above < uint32_t(k) && uint32_t(k) <= above + c[i]) {
+        s_misc[0] = lane * 8 + i;
+        s_misc[1] = static_cast<int>(above);
+        s_misc[2] = static_cast<int>(c[i]);
+      }
+      above += c[i];
+    }
+    if (lane == 0) s_misc[3] = 0;
+  }
+  compute_sync();
+  const int bstar = s_misc[0], n_above = s_misc[1], nb = s_misc[2];
+  if (nb > kCT) return false;
+  for (int j = tid; j < n; j += kCT) {
+    const int bin = value_bin(vals[j], lo, scale);
+    if (bin == bstar) cand[atomicAdd(&s_misc[3], 1)] = j;
+    flag[j] = bin > bstar;
+  }
+  compute_sync();
+  if (tid < nb) {
+    const int j = cand[tid];
+    const float x = vals[j];
+    int rank = 0;  // boundary-bin members ahead of j
+    for (int m = 0; m < nb; ++m) {
+      const int jm = cand[m];
+      const float y = vals[jm];
+      rank += y > x || (y == x && jm < j);
+    }
+    flag[j] = rank < k - n_above;
+  }
+  compute_sync();
+  write_selected(a, bh, flag, s_w);
+  compute_sync();
+  return true;
+}
+
+// Top-k of row bh into idx[bh], ascending (compute warps; ends with a barrier).
+__device__ __forceinline__ void select_row(const FusedArgs& a, int bh, uint32_t* hist, int* s_w,
+                                           int* s_misc, float* s_f, uint32_t* keys,
+                                           uint8_t* flag, int* cand) {
+  const int n = a.at.nc, k = a.at.k;
+  if (k >= n) {  // every candidate
+    for (int j = ctid(); j < n; j += kCT) a.idx[int64_t(bh) * k + j] = a.at.first + j;
+    compute_sync();
+    return;
+  }
+  if (!topk_binned(a, bh, hist, s_w, s_misc, s_f, reinterpret_cast<float*>(keys), flag, cand))
+    topk_radix(a, bh, hist, s_w, s_misc, keys, flag);
+}
+
+// ---------------------------------------------------------------------------
+// staging (warp 0)
+
+// Stages one item into `stg`: bulk copies that complete on `bar`, whose
+// transaction count is armed with the item's bytes.  Selected rows wait
+// (bounded) for the head's selection.  False: aborting or timed out, nothing
+// armed.
 template <typename T, int D>
-__device__ int issue_item(const FusedArgs& a, const Item& item, char* stg, uint64_t* bar,
-                          Meta* meta, int* sel_pref, int* sel_phys, int* sel_bh, bool may_wait) {
-  using C = DecodeTile<T, D>;
+__device__ bool issue_item(const FusedArgs& a, const Item& item, char* stg, uint64_t* bar,
+                           Meta* meta, int* sel_pref, int* sel_phys, int* sel_bh,
+                           volatile int* abort_flag) {
+  using C = DecodeTile<T, D, kCW>;
   const int lane = threadIdx.x & 31;
   if (item.kind == 0) {
     const int n = item.v1 - item.v0;
@@ -411,7 +573,7 @@ __device__ int issue_item(const FusedArgs& a, const Item& item, char* stg, uint6
                bytes, bar);
     }
     __syncwarp();
-    return 1;
+    return true;
   }
   const int* pref;
   const int* phys;
@@ -428,29 +590,26 @@ __device__ int issue_item(const FusedArgs& a, const Item& item, char* stg, uint6
     nseg = 2;
   } else {
     if (item.bh != *sel_bh) {
-      // this head's selection (lane 0 polls), then the layout of its blocks
-      int ok = 0;
-      if (lane == 0) {
-        const uint32_t* flag = a.ready + item.bh;
-        ok = ld_acquire(flag) != 0;
-        if (!ok && may_wait) {
-          const unsigned long long t0 = now_ns();
-          while (!(ok = ld_acquire(flag) != 0)) {
-            __nanosleep(64);
-            if (now_ns() - t0 > kTimeoutNs) break;
+      // this head's selection (every lane acquires the flag), then the
+      // layout of its blocks
+      const uint32_t* flag = a.ready + item.bh;
+      bool ok = ld_acquire(flag) != 0;
+      if (!__all_sync(0xffffffffu, ok)) {
+        const unsigned long long t0 = now_ns();
+        while (true) {
+          __nanosleep(32);
+          if (!ok) ok = ld_acquire(flag) != 0;
+          if (__all_sync(0xffffffffu, ok)) break;
+          if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
+          if (__shfl_sync(0xffffffffu, now_ns() - t0 > kTimeoutNs, 0)) {
+            if (lane == 0) {
+              report(a.at.status, RBA_ERR_TIMEOUT, kWhereFused, 2);
+              *abort_flag = 1;
+            }
+            __syncwarp();
+            return false;
           }
         }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok && !may_wait) return 0;
-      if (!ok) {
-        if (lane == 0) {
-          report(a.at.status, RBA_ERR_TIMEOUT, kWhereFused, 2);
-          meta->nrows = 0;
-          mbar_arrive_tx(bar, 0);
-        }
-        __syncwarp();
-        return -1;
       }
       const int k = a.at.k;
       int run = 0;
@@ -514,7 +673,38 @@ __device__ int issue_item(const FusedArgs& a, const Item& item, char* stg, uint6
     }
   }
   __syncwarp();
-  return 1;
+  return true;
+}
+
+// Warp 0: stage every item of this CTA, in order, into the stage ring.
+template <typename T, int D>
+__device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64_t* full,
+                                        uint64_t* empty, Meta* meta, int* sel_pref,
+                                        int* sel_phys, volatile int* abort_flag,
+                                        const int64_t* B0, const int64_t* B1) {
+  using C = DecodeTile<T, D, kCW>;
+  const int NS = a.NS;
+  Iter it;
+  iter_begin(a, it, B0);
+  Item item;
+  int j = 0, s = 0, sel_bh = -1;
+  uint32_t ph = 0;  // phase parity of the stage's next fill
+  while (next_item<C::TT>(a, it, item, B1)) {
+    // stage s is free once every compute warp released its previous item
+    if (j >= NS && !mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.at.status, 1)) break;
+    if (!issue_item<T, D>(a, item, stages + size_t(s) * C::STAGE, &full[s], &meta[s], sel_pref,
+                          sel_phys, &sel_bh, abort_flag))
+      break;
+    ++j;
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  // no copy may still be landing in shared memory when the CTA exits
+  if ((threadIdx.x & 31) == 0)
+    for (int q = max(0, j - NS); q < j; ++q) mbar_drain(&full[q % NS], (q / NS) & 1u);
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
@@ -522,7 +712,7 @@ __device__ int issue_item(const FusedArgs& a, const Item& item, char* stg, uint6
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
-  using C = DecodeTile<T, D>;
+  using C = DecodeTile<T, D, kCW>;
   using S = FusedSmem<T, D, G>;
   extern __shared__ __align__(128) char smem[];
   const int NS = a.NS;
@@ -532,161 +722,127 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   int* sel_phys = sel_pref + (kMaxK + 1);
   float* wslot = reinterpret_cast<float*>(reinterpret_cast<char*>(sel_pref) + S::SEL);
   char* misc = reinterpret_cast<char*>(wslot) + S::SLOTS;
-  uint64_t* full = reinterpret_cast<uint64_t*>(misc);               // [4]
-  uint64_t* empty = full + kMaxStages;                              // [4]
-  Meta* meta = reinterpret_cast<Meta*>(empty + kMaxStages);         // [4]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(meta + kMaxStages);  // [256]
-  int* s_w = reinterpret_cast<int*>(hist + 256);                    // [32]
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);               // [kMaxStages]
+  uint64_t* empty = full + kMaxStages;                              // [kMaxStages]
+  Meta* meta = reinterpret_cast<Meta*>(empty + kMaxStages);         // [kMaxStages]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(meta + kMaxStages);  // [kBins + 1]
+  int* s_w = reinterpret_cast<int*>(hist + kBins + 1);              // [32]
   int* s_misc = s_w + 32;                                           // [16]
   int* owned = s_misc + 16;                                         // [kMaxTouch]
   volatile int* abort_flag = owned + kMaxTouch;                     // [4]
-  float* qsum_s = reinterpret_cast<float*>(owned + kMaxTouch + 4);  // [D]
-  uint32_t* topk_buf = reinterpret_cast<uint32_t*>(misc + S::MISC);        // [kMaxN]
-  int64_t* B0 = reinterpret_cast<int64_t*>(misc + S::MISC + S::KEYS);      // [P+1] candidates
-  int64_t* B1 = B0 + (kMaxGrid + 1);                                       // [P+1] attention
+  float* s_f = reinterpret_cast<float*>(owned + kMaxTouch + 4);     // [32]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(misc + S::MISC);     // [kMaxN]
+  uint8_t* flag = reinterpret_cast<uint8_t*>(misc + S::MISC + S::KEYS);  // [kMaxN]
+  int* cand = reinterpret_cast<int*>(flag + kMaxN);                      // [kCT]
+  int64_t* B0 = reinterpret_cast<int64_t*>(misc + S::MISC + S::KEYS + S::FLAGS);  // candidates
+  int64_t* B1 = B0 + (kMaxGrid + 1);                                              // attention
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int P = gridDim.x, p = blockIdx.x;
   const int64_t Lh = int64_t(a.L_st) + a.U_sel;
-  if (tid == 0) {
+  if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCW);
     }
     *abort_flag = 0;
-    s_misc[15] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  for (int q = tid; q <= P; q += kFT) {
+  for (int q = threadIdx.x; q <= P; q += kFT) {
     B0[q] = bnd(q, P, int64_t(a.at.k > 0 ? a.at.nc : 0) * a.BH);
     B1[q] = bnd(q, P, Lh * a.BH);
   }
   __syncthreads();
+  if (warp == 0) {
+    produce<T, D>(a, stages, full, empty, meta, sel_pref, sel_phys, abort_flag, B0, B1);
+    return;
+  }
+  // ---- compute warps from here on (named barrier 1; no __syncthreads)
+  const int cw = warp - 1, tid = ctid();
 
-  // ---- staging by warp 0: item j goes to stage j % NS once every warp has
-  // released item j - NS (empty barrier).  Selected rows are not staged
-  // before this CTA has published its own selections; a head whose selection
-  // is not out, or a stage not yet released, is only waited for when the
-  // item is the one needed now (index cur).
-  Iter pit;
-  iter_begin(a, pit, B0, B1);
-  Item pnext;
-  bool have_pnext = next_item<C::TT>(a, pit, pnext, B1);
-  int issued = 0, sel_bh = -1;
-  bool scores_done = false;
-  auto issue_ahead = [&](int cur) {
-    if (warp != 0) return;
-    while (have_pnext && issued <= cur + NS - 1 && !(pnext.kind == 2 && !scores_done)) {
-      const int s = issued % NS;
-      const bool now = issued <= cur;
-      if (issued >= NS && !*abort_flag) {
-        const uint32_t par = ((issued / NS) - 1) & 1u;
-        if (!now && !mbar_try(&empty[s], par)) break;
-        if (now && !mbar_wait(&empty[s], par)) {
-          if (lane == 0) report(a.at.status, RBA_ERR_TIMEOUT, kWhereFused, 1);
-          *abort_flag = 1;
-        }
-      }
-      // 1 staged, 0 not yet (stop for now), -1 timed out (armed empty), 2 skipped
-      int r = 2;
-      if (!*abort_flag)
-        r = issue_item<T, D>(a, pnext, stages + size_t(s) * C::STAGE, &full[s], &meta[s],
-                             sel_pref, sel_phys, &sel_bh, now);
-      if (r == 0) break;
-      if (r < 0) *abort_flag = 1;
-      if (r == 2 && lane == 0) {  // after an abort: arm the stage with no copy
-        meta[s].nrows = 0;
-        mbar_arrive_tx(&full[s], 0);
-      }
-      __syncwarp();
-      ++issued;
-      have_pnext = next_item<C::TT>(a, pit, pnext, B1);
-    }
-    if (lane == 0) s_misc[15] = issued;
-  };
-  // wait for item i's data; after an abort, items are skipped (no wait)
-  auto wait_item = [&](int i) -> bool {
-    issue_ahead(i);
-    const int s = i % NS;
-    if (*abort_flag) return false;
-    if (!mbar_wait(&full[s], (i / NS) & 1u)) {
-      if (lane == 0) report(a.at.status, RBA_ERR_TIMEOUT, kWhereFused, 3);
-      *abort_flag = 1;
-      return false;
-    }
-    return true;
-  };
-  auto release_item = [&](int i) {
+  // item i of this CTA sits in stage s with parity ph
+  int s = 0;
+  uint32_t ph = 0;
+  auto wait_full = [&]() -> bool { return mbar_wait(&full[s], ph, abort_flag, a.at.status, 3); };
+  auto release = [&]() {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[i % NS]);
+    if (lane == 0) mbar_arrive(&empty[s]);
+  };
+  auto advance = [&]() {
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1u;
+    }
   };
 
-  issue_ahead(-1);
+  // summed query of every head this CTA scores (GQA: the group's q heads)
+  const int64_t sr0 = B0[p], sr1 = B0[p + 1];
+  const int bh_first = sr1 > sr0 ? static_cast<int>(sr0 / a.at.nc) : 0;
+  const int n_touch = sr1 > sr0 ? static_cast<int>((sr1 - 1) / a.at.nc) - bh_first + 1 : 0;
+  float* qsum = reinterpret_cast<float*>(keys);  // [n_touch][D]
+  for (int x = tid; x < n_touch * D; x += kCT) {
+    const int bh = bh_first + x / D, d = x % D;
+    const int b = bh / a.at.Hkv, h = bh % a.at.Hkv;
+    const T* qp = static_cast<const T*>(a.at.q) + (int64_t(b) * a.at.Hq + h * G) * D + d;
+    float qs = 0.f;
+    for (int gg = 0; gg < G; ++gg) qs += Elem<T>::to_f32(qp[gg * D]);
+    qsum[x] = qs;
+  }
+  compute_sync();
+
   Iter it;
-  iter_begin(a, it, B0, B1);
+  iter_begin(a, it, B0);
   Item item;
   bool have = next_item<C::TT>(a, it, item, B1);
-  int i = 0;
 
   // ---- phase 1: score this CTA's candidates
-  int qsum_bh = -1;
   while (have && item.kind == 0) {
-    const bool ok = wait_item(i);
-    const char* stg = stages + size_t(i % NS) * C::STAGE;
-    const int nrows = ok ? meta[i % NS].nrows : 0;
-    const int bh = item.bh;
-    if (bh != qsum_bh) {  // the group's summed query, once per head
-      compute_sync();
-      const int b = bh / a.at.Hkv, h = bh % a.at.Hkv;
-      const T* qp = static_cast<const T*>(a.at.q) + (int64_t(b) * a.at.Hq + h * G) * D;
-      for (int d = tid; d < D; d += kCT) {
-        float qs = 0.f;
-        for (int gg = 0; gg < G; ++gg) qs += Elem<T>::to_f32(qp[gg * D + d]);
-        qsum_s[d] = qs;
-      }
-      compute_sync();
-      qsum_bh = bh;
-    }
-    const int vpc = a.rep_bytes / 16;     // vectors per candidate
-    const int lpc = vpc < 32 ? vpc : 32;  // lanes per candidate
-    const int cpw = 32 / lpc;
-    const int sub = lane % lpc, slot = lane / lpc;
-    for (int c = warp * cpw + slot; c - slot < nrows; c += kCW * cpw) {
-      float acc = 0.f;
-      if (c < nrows) {
-        for (int v = sub; v < vpc; v += lpc) {
-          const uint4 u = *reinterpret_cast<const uint4*>(stg + size_t(c) * a.rep_bytes + v * 16);
-          float f[8];
-          if (a.rep_f32) {
-            const int d0 = (v * 4) % D;
-            unpack(u, f, 0.f);
-            const float4 qv = *reinterpret_cast<const float4*>(qsum_s + d0);
-            acc = fmaf(qv.x, f[0], acc);
-            acc = fmaf(qv.y, f[1], acc);
-            acc = fmaf(qv.z, f[2], acc);
-            acc = fmaf(qv.w, f[3], acc);
-          } else {
-            const int d0 = (v * 8) % D;
-            unpack(u, f, __nv_bfloat16());
-            const float4 q0 = *reinterpret_cast<const float4*>(qsum_s + d0);
-            const float4 q1 = *reinterpret_cast<const float4*>(qsum_s + d0 + 4);
-            acc = fmaf(q0.x, f[0], acc);
-            acc = fmaf(q0.y, f[1], acc);
-            acc = fmaf(q0.z, f[2], acc);
-            acc = fmaf(q0.w, f[3], acc);
-            acc = fmaf(q1.x, f[4], acc);
-            acc = fmaf(q1.y, f[5], acc);
-            acc = fmaf(q1.z, f[6], acc);
-            acc = fmaf(q1.w, f[7], acc);
+    if (wait_full()) {
+      const char* stg = stages + size_t(s) * C::STAGE;
+      const int nrows = meta[s].nrows;
+      const float* qv_ = qsum + (item.bh - bh_first) * D;
+      const int vpc = a.rep_bytes / 16;     // vectors per candidate
+      const int lpc = vpc < 32 ? vpc : 32;  // lanes per candidate
+      const int cpw = 32 / lpc;
+      const int sub = lane % lpc, slot = lane / lpc;
+      for (int c = cw * cpw + slot; c - slot < nrows; c += kCW * cpw) {
+        float acc = 0.f;
+        if (c < nrows) {
+          for (int v = sub; v < vpc; v += lpc) {
+            const uint4 u =
+                *reinterpret_cast<const uint4*>(stg + size_t(c) * a.rep_bytes + v * 16);
+            float f[8];
+            if (a.rep_f32) {
+              const int d0 = (v * 4) % D;
+              unpack(u, f, 0.f);
+              const float4 qv = *reinterpret_cast<const float4*>(qv_ + d0);
+              acc = fmaf(qv.x, f[0], acc);
+              acc = fmaf(qv.y, f[1], acc);
+              acc = fmaf(qv.z, f[2], acc);
+              acc = fmaf(qv.w, f[3], acc);
+            } else {
+              const int d0 = (v * 8) % D;
+              unpack(u, f, __nv_bfloat16());
+              const float4 q0 = *reinterpret_cast<const float4*>(qv_ + d0);
+              const float4 q1 = *reinterpret_cast<const float4*>(qv_ + d0 + 4);
+              acc = fmaf(q0.x, f[0], acc);
+              acc = fmaf(q0.y, f[1], acc);
+              acc = fmaf(q0.z, f[2], acc);
+              acc = fmaf(q0.w, f[3], acc);
+              acc = fmaf(q1.x, f[4], acc);
+              acc = fmaf(q1.y, f[5], acc);
+              acc = fmaf(q1.z, f[6], acc);
+              acc = fmaf(q1.w, f[7], acc);
+            }
           }
         }
+        for (int o = lpc / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (sub == 0 && c < nrows) a.scores[int64_t(item.bh) * a.at.nc + item.v0 + c] = acc;
       }
-      for (int o = lpc / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (sub == 0 && c < nrows) a.scores[int64_t(bh) * a.at.nc + item.v0 + c] = acc;
+      release();
     }
-    release_item(i);
-    ++i;
+    advance();
     have = next_item<C::TT>(a, it, item, B1);
   }
 
@@ -694,13 +850,12 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   compute_sync();
   if (tid == 0) {
     int n_owned = 0;
-    const int64_t r0 = B0[p], r1 = B0[p + 1];
-    if (r1 > r0) {
+    if (sr1 > sr0) {
       const int64_t L = a.at.nc;
-      for (int bh = static_cast<int>(r0 / L); bh <= static_cast<int>((r1 - 1) / L); ++bh) {
-        const int64_t s0 = max(r0, bh * L), s1 = min(r1, (bh + 1) * L);
-        const uint32_t cnt = static_cast<uint32_t>(s1 - s0);
-        const uint32_t old = atom_add_acq_rel(a.score_cnt + bh, cnt);
+      for (int bh = bh_first; bh < bh_first + n_touch; ++bh) {
+        const int64_t c0 = max(sr0, bh * L), c1 = min(sr1, (bh + 1) * L);
+        const uint32_t cnt = static_cast<uint32_t>(c1 - c0);
+        const uint32_t old = atom_add_acq_rel(a.score_cnt + bh, cnt);  // publishes our scores
         if (old + cnt == uint32_t(a.at.nc) && n_owned < kMaxTouch) owned[n_owned++] = bh;
       }
     }
@@ -709,13 +864,12 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   compute_sync();
   for (int o = 0; o < s_misc[8]; ++o) {
     const int bh = owned[o];
-    topk_row(a, bh, hist, s_w, s_misc, topk_buf);  // ends with a barrier
+    select_row(a, bh, hist, s_w, s_misc, s_f, keys, flag, cand);  // ends with a barrier
     if (tid == 0) {
       __threadfence();
       st_release(a.ready + bh, 1u);
     }
   }
-  scores_done = true;
 
   // ---- attention over this CTA's rows, head by head
   LaneState<T, D, G> st;
@@ -723,7 +877,7 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   float* m_s = wslot + kMaxSlots;               // [nl][G]
   float* l_s = m_s + G * kMaxSlots;             // [nl][G]
   float* w_s = l_s + G * kMaxSlots;             // [G][nl]
-  int* list = reinterpret_cast<int*>(wslot);    // [nl]
+
   while (true) {
     const bool more = have;
     if (cur_bh >= 0 && (!more || item.bh != cur_bh)) {
@@ -735,7 +889,7 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
       if (slot_lane == 0) {
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
-          float* r = red + (warp * G + gg) * (D + 2);
+          float* r = red + (cw * G + gg) * (D + 2);
           if (part == 0) {
             r[0] = st.m[gg];
             r[1] = st.l[gg];
@@ -790,8 +944,8 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
           l_s[x] = __ldcg(sp + 1);
         }
         compute_sync();
-        if (warp < G) {
-          const int gg = warp;
+        if (cw < G) {
+          const int gg = cw;
           float M = -INFINITY;
           for (int j = lane; j < nl; j += 32) M = fmaxf(M, m_s[j * G + gg]);
           for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -818,7 +972,7 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
 #pragma unroll
         for (int e = 0; e < PER; ++e) acc[e] = 0.f;
 #pragma unroll 1
-        for (int j = warp; j < nl; j += kCW) {
+        for (int j = cw; j < nl; j += kCW) {
           const float* sp = base + int64_t(j) * G * (D + 2);
           float v[PER];
 #pragma unroll
@@ -835,7 +989,7 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
 #pragma unroll
         for (int e = 0; e < PER; ++e) {
           const int x = lane + 32 * e;
-          if (x < G * D) red[warp * G * D + x] = acc[e];
+          if (x < G * D) red[cw * G * D + x] = acc[e];
         }
         compute_sync();
         for (int x = tid; x < G * D; x += kCT) {
@@ -859,15 +1013,12 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
       cur_bh = item.bh;
       load_q<T, D, G>(a.at, cur_bh, st);
     }
-    if (wait_item(i)) consume_tile<T, D, G>(stages + size_t(i % NS) * C::STAGE, meta[i % NS].nrows, st);
-    release_item(i);
-    ++i;
+    if (wait_full()) {
+      consume_tile<T, D, G, kCW>(stages + size_t(s) * C::STAGE, meta[s].nrows, st, cw);
+      release();
+    }
+    advance();
     have = next_item<C::TT>(a, it, item, B1);
-  }
-  // drain (bounded): no copy may still be landing in shared memory at exit
-  if (*abort_flag && warp == 0) {
-    const int n_issued = s_misc[15];
-    for (int j = max(0, n_issued - NS); j < n_issued; ++j) mbar_wait(&full[j % NS], (j / NS) & 1u);
   }
 }
 
@@ -875,7 +1026,7 @@ template <typename T, int D, int G>
 int fused_stages() {
   using S = FusedSmem<T, D, G>;
   int NS = kMaxStages;
-  while (NS > 2 && S::bytes(NS) > 220 * 1024) --NS;
+  while (NS > 2 && S::bytes(NS) > 227 * 1024) --NS;
   return NS;
 }
 
@@ -907,7 +1058,7 @@ int fused_occupancy_t() {
 template <typename T, int D, int G>
 rba_status launch_fused_t(FusedArgs a, int P, cudaStream_t stream) {
   using S = FusedSmem<T, D, G>;
-  using C = DecodeTile<T, D>;
+  using C = DecodeTile<T, D, kCW>;
   const int NS = fused_stages<T, D, G>();
   a.NS = NS;
   a.score_cap = C::STAGE / a.rep_bytes;

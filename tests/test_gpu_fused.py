@@ -52,3 +52,39 @@ def test_fused_step_equals_three_launches(rba, name):
         err = float((out - out3).abs().max()) / vmax
         assert err <= OUT_TOL[w.dtype], (rep, err)
         assert float((lse - lse3).abs().max()) <= OUT_TOL[w.dtype]
+
+
+@pytest.mark.parametrize("n_distinct", [1, 2, 3, 40])
+def test_fused_selection_with_tied_scores(rba, n_distinct):
+    # Landmark keys drawn from n_distinct vectors: scores repeat exactly, so
+    # the k-th largest value is shared by many candidates and the tie goes to
+    # the lowest block ids.  With ~650 candidates, 3 values leave ~220 tied
+    # candidates at the boundary (exact ranking inside the boundary value
+    # bin), 2 values ~325 (more than the in-bin ranking takes: radix select),
+    # 1 value a zero score range (radix select).
+    w = W["landmark-decode-b16"].scaled(batch=2, n_q_heads=4, n_kv_heads=4, top_k=9)
+    x = synth.decode_inputs(w)
+    rng = np.random.default_rng(11)
+    lm = x["landmarks"].copy()
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            lm[b, h] = x["landmarks"][b, h, rng.integers(0, n_distinct, w.n_blocks)]
+    x = dict(x, landmarks=lm)
+    st = make_decode_store(rba, w, x)
+    q = dev(x["q"], w.dtype)
+    first, nc = st.candidates(w.context, w.sink, w.window)
+    scores = st.score(q, w.context, w.sink, w.window)
+    idx3 = rba.topk(scores.reshape(-1, nc), w.top_k, index_base=first).reshape(
+        w.batch, w.n_kv_heads, w.top_k)
+    out3, _ = st.attend(q, idx3, w.context, w.sink, w.window)
+    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 1
+    idx, out, _ = st.decode_step(q, w.top_k, w.context, w.sink, w.window)
+    st.check()
+    assert torch.equal(idx, idx3)
+    # ties really go to the lowest ids: brute force on the GPU's own scores
+    s = scores.reshape(w.batch * w.n_kv_heads, nc).cpu().numpy()
+    for r in range(s.shape[0]):
+        order = sorted(range(nc), key=lambda j: (-s[r, j], j))[:w.top_k]
+        assert idx.reshape(-1, w.top_k)[r].tolist() == [first + j for j in sorted(order)]
+    vmax = float(st.v.float().abs().max())
+    assert float((out - out3).abs().max()) / vmax <= OUT_TOL[w.dtype]
