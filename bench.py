@@ -64,6 +64,10 @@ def parse(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="bound on the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-config measurements (other decode configs, prefill)")
+    ap.add_argument("--config-seconds", type=float, default=0.5,
+                    help="timed GPU seconds per extra config")
     ap.add_argument("--workload", default=WORKLOAD, help=argparse.SUPPRESS)
     ap.add_argument("--replicas", type=int, default=0, help=argparse.SUPPRESS)
     return ap.parse_args(argv)
@@ -232,6 +236,17 @@ def count_kernel_nodes(graph):
         return kinds
     except Exception:
         return None
+
+
+def prefill_pairs(w, idx):
+    """(query, key) pairs a prefill step attends: every row of a chunk sees the
+    retrieved past tokens of its selection and its own chunk causally.
+    idx: [n_chunks][n_sel][k] (n_sel = 1: one selection shared by all heads)."""
+    counts = attended_counts(idx, w.context, w.block_size, w.sink, w.window)
+    heads_per_sel = w.n_q_heads if idx.shape[1] == 1 else w.n_q_heads // w.n_kv_heads
+    past = int(counts.sum()) * heads_per_sel * w.chunk_len
+    own = w.n_chunks * w.n_q_heads * w.chunk_len * (w.chunk_len + 1) // 2
+    return past + own
 
 
 # ---------------------------------------------------------------------------
@@ -445,6 +460,10 @@ def run_ours(args):
                "d2h_bytes_per_step": out_h.numel() * 4 + lse_h.numel() * 4 + idx_h.numel() * 4,
                "steps": args.e2e_steps, "call": "rba_decode_step_host (pinned host buffers)"}
 
+    configs = None
+    if world == 1 and not args.no_configs:
+        configs = measure_configs(dev, args.config_seconds)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, x, args.cpu_seconds, args.workload)
@@ -488,8 +507,224 @@ def run_ours(args):
         "graph_kernel_nodes_per_step": n_nodes,
         "path": "fused single launch" if plan == 1 else f"three launches (plan {plan})",
         "cpu_baseline": cpu,
+        "configs": configs,
     }
     return line
+
+
+def _to_dev(a, dtype, dev):
+    import torch
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+
+
+def _time_graph(g, stream, seconds, min_iters=5):
+    """Average ms per replay of CUDA graph g, over about `seconds` of replays."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        e0.record(stream)
+        for _ in range(min_iters):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    est = e0.elapsed_time(e1) / min_iters
+    n = max(min_iters, int(seconds * 1e3 / max(est, 1e-3)))
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n, n
+
+
+def measure_decode_config(name, dev, seconds, pk):
+    """Decode-step throughput of one decode config (graph-replayed steps; L2
+    defeated by rotating store replicas, or by an L2-sized write between
+    steps whose own time is subtracted when replicas would not fit)."""
+    import torch
+    import retrieval_block_sparse_b200 as rba
+    from retrieval_block_sparse_b200 import synth
+    w = synth.WORKLOADS[name]
+    x = synth.decode_inputs(w)
+
+    def new_store():
+        return rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                         head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
+                         dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep, device=dev)
+    st = new_store()
+    st.k.copy_(_to_dev(x["K"], w.dtype, dev))
+    st.v.copy_(_to_dev(x["V"], w.dtype, dev))
+    aux = None
+    if w.rep_mode == "topr_attn":
+        aux = _to_dev(x["probe"], w.dtype, dev)
+    elif w.rep_mode == "external":
+        aux = _to_dev(x["landmarks"], w.dtype, dev).reshape(w.batch, w.n_kv_heads, w.n_blocks,
+                                                             1, w.head_dim)
+    if w.rep_mode != "identity":
+        st.memorize(None, None, first_block=0, n_blocks=w.n_blocks, aux=aux)
+    del x["K"], x["V"]
+    q = _to_dev(x["q"], w.dtype, dev)
+    first, nc = st.candidates(w.context, w.sink, w.window)
+    idx0, _, _ = st.decode_step(q, w.top_k, w.context, w.sink, w.window)
+    st.check()
+    rep_b, gath_b = step_bytes(w, nc, idx0.cpu().numpy())
+    nbytes = rep_b + gath_b
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    store_bytes = st.k.numel() * st.k.element_size() * 2 + (
+        st.rep.numel() * st.rep.element_size() if st.rep is not None else 0)
+    R = max(1, math.ceil(4 * l2 / nbytes))
+    use_flush = R > 16 or R * store_bytes > 48e9
+    stores = [st]
+    if not use_flush:
+        for _ in range(R - 1):
+            s2 = new_store()
+            s2.k.copy_(st.k)
+            s2.v.copy_(st.v)
+            if st.rep is not None:
+                s2.rep.copy_(st.rep)
+            stores.append(s2)
+    ws = [s.decode_workspace(w.top_k, w.context, w.sink, w.window) for s in stores]
+    outs = [torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+            for _ in stores]
+    lses = [torch.empty((w.batch, w.n_q_heads), dtype=torch.float32, device=dev)
+            for _ in stores]
+    idxs = [torch.empty((w.batch, w.n_kv_heads, w.top_k), dtype=torch.int32, device=dev)
+            for _ in stores]
+    flush = torch.empty(max(4 * l2, 1 << 20), dtype=torch.uint8, device=dev) if use_flush \
+        else None
+
+    def step(r):
+        stores[r].decode_step(q, w.top_k, w.context, w.sink, w.window, workspace=ws[r],
+                              out=outs[r], lse=lses[r], idx=idxs[r])
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for r in range(len(stores)):
+            step(r)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for r in range(len(stores)):
+            if use_flush:
+                flush.fill_(1)
+            step(r)
+    ms, n = _time_graph(g, stream, seconds)
+    ms /= len(stores)
+    if use_flush:
+        gf = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gf, stream=stream):
+            flush.fill_(1)
+        ms_f, _ = _time_graph(gf, stream, seconds / 4)
+        ms -= ms_f
+    for s in stores:
+        s.check()
+    us = ms * 1e3
+    gbs = nbytes / (us * 1e-6) / 1e9
+    plan = st.decode_plan(w.top_k, w.context, w.sink, w.window)
+    return {"workload": name, "steps_per_s": round(1e6 / us, 2), "us_per_step": round(us, 3),
+            "algorithmic_bytes": nbytes, "rep_key_bytes": rep_b, "gathered_kv_bytes": gath_b,
+            "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
+            "path": "fused single launch" if plan == 1 else "three launches",
+            "steps_timed": n * len(stores),
+            "l2": (f"L2-sized write between steps, its time subtracted" if use_flush else
+                   f"{len(stores)} store replicas rotated ({len(stores)} x {nbytes / 1e6:.1f} MB"
+                   f" >= 4 x L2)")}
+
+
+def measure_prefill_config(name, dev, seconds, pk):
+    """Chunked-prefill step of one prefill config: selection (score + top-k)
+    and the retrieval-causal tensor-core attention, timed apart."""
+    import torch
+    import retrieval_block_sparse_b200 as rba
+    from retrieval_block_sparse_b200 import synth
+    w = synth.WORKLOADS[name]
+    x = synth.prefill_inputs(w)
+    mode = "embed_cosine" if w.score_mode == "cosine" else (
+        "identity" if w.block_size == 1 else "mean")
+    st = rba.Store(batch=1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
+                   block_size=w.block_size, capacity_tokens=w.context, dtype=w.dtype, mode=mode,
+                   d_ret=w.d_ret, device=dev)
+    st.k.copy_(_to_dev(x["K"], w.dtype, dev))
+    st.v.copy_(_to_dev(x["V"], w.dtype, dev))
+    del x["K"], x["V"]
+    nb = w.context // w.block_size
+    if mode == "embed_cosine":
+        st.memorize(None, None, first_block=0, n_blocks=nb,
+                    aux=torch.from_numpy(x["bank_embed"]).to(dev).reshape(1, nb, w.d_ret))
+    elif mode == "mean":
+        st.memorize(None, None, first_block=0, n_blocks=nb)
+    Q = _to_dev(x["Q"], w.dtype, dev)
+    Kc, Vc = _to_dev(x["chunk_K"], w.dtype, dev), _to_dev(x["chunk_V"], w.dtype, dev)
+    first, nc = st.candidates(w.context, w.sink, w.window)
+    qsel = torch.from_numpy(x["query_embed"]).to(dev) if mode == "embed_cosine" else Q
+    n_sel = 1 if mode == "embed_cosine" else w.n_kv_heads
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    sc = st.score(qsel, w.context, w.sink, w.window)
+    idx = rba.topk(sc.reshape(-1, nc), w.top_k, index_base=first).reshape(w.n_chunks, n_sel,
+                                                                           w.top_k)
+    out = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+    lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+    ws = st.prefill_workspace(w.n_chunks, w.chunk_len, n_sel, w.top_k, w.context, w.sink,
+                              w.window)
+    rows = sc.numel() // nc
+    topk_ws = torch.empty(max(rba.lib().rba_topk_workspace_size(rows, nc, w.top_k), 16),
+                          dtype=torch.uint8, device=dev)
+
+    def select():
+        st.score(qsel, w.context, w.sink, w.window, out=sc)
+        rba.topk(sc.reshape(-1, nc), w.top_k, index_base=first, out=idx.reshape(-1, w.top_k),
+                 workspace=topk_ws)
+
+    def attend():
+        st.attend_prefill(Q, idx, Kc, Vc, w.context, w.sink, w.window, out=out, lse=lse,
+                          workspace=ws)
+    with torch.cuda.stream(stream):
+        select()
+        attend()
+    torch.cuda.synchronize()
+    st.check()
+    gs, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gs, stream=stream):
+        select()
+    with torch.cuda.graph(ga, stream=stream):
+        attend()
+    ms_s, _ = _time_graph(gs, stream, seconds / 2)
+    ms_a, n_a = _time_graph(ga, stream, seconds)
+    st.check()
+    pairs = prefill_pairs(w, idx.cpu().numpy())
+    flops = 4 * w.head_dim * pairs
+    tflops = flops / (ms_a * 1e-3) / 1e12
+    scan = None if mode == "embed_cosine" else (
+        w.n_kv_heads * nc * w.head_dim * 2 if mode == "identity" else
+        w.n_kv_heads * nc * w.head_dim * 4)
+    del topk_ws
+    res = {"workload": name, "attend_us": round(ms_a * 1e3, 2), "attend_calls_timed": n_a,
+           "pairs": pairs, "flops": flops, "attend_tflops": round(tflops, 1),
+           "attend_frac_of_bf16_peak": round(tflops / pk["bf16_tflops"], 4),
+           "bf16_peak_tflops": pk["bf16_tflops"], "select_us": round(ms_s * 1e3, 2),
+           "l2": "inputs larger than L2 (K/V of the retrieved set + chunk + Q)"}
+    if scan is not None:
+        res["select_scan_bytes"] = scan
+        res["select_gbs"] = round(scan / (ms_s * 1e-3) / 1e9, 1)
+        res["select_frac_of_hbm"] = round(scan / (ms_s * 1e-3) / 1e9 / pk["hbm_gbs"], 4)
+    return res
+
+
+def measure_configs(dev, seconds):
+    pk = peaks()
+    out = {}
+    for name in ("tiny-decode-f32", "landmark-decode-b16", "token-retrieval-decode-1m"):
+        out[name] = measure_decode_config(name, dev, seconds, pk)
+    for name in ("memlong-cosine-prefill", "token-retrieval-prefill-1m"):
+        out[name] = measure_prefill_config(name, dev, seconds, pk)
+    return out
 
 
 # ---------------------------------------------------------------------------

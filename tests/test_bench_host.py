@@ -68,3 +68,34 @@ def test_reference_arm_line():
     assert line["unit"] == bench.UNIT and line["metric"] == bench.METRIC
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+
+
+def test_prefill_pairs_match_brute_force_and_published_sizes():
+    from retrieval_block_sparse_b200 import synth
+    W = synth.WORKLOADS
+    # brute force on a tiny case: count (row, key) pairs of the oracle's own
+    # attended-token rule (past set per selection) plus the causal chunk
+    w = W["token-retrieval-prefill-1m"].scaled(n_chunks=2, n_q_heads=4, n_kv_heads=2,
+                                               chunk_len=5, context=200, block_size=10,
+                                               sink=7, window=23, top_k=3)
+    rng = np.random.default_rng(0)
+    first = w.sink // w.block_size
+    nc = -(-(w.context - w.window) // w.block_size) - first
+    idx = np.stack([np.stack([np.sort(rng.choice(nc, 3, replace=False)) + first
+                              for _ in range(w.n_kv_heads)]) for _ in range(w.n_chunks)])
+    brute = 0
+    for c in range(w.n_chunks):
+        for hq in range(w.n_q_heads):
+            toks = O.attended_tokens(w.context, w.block_size, w.sink, w.window,
+                                     idx[c, hq // (w.n_q_heads // w.n_kv_heads)])
+            for i in range(w.chunk_len):
+                brute += len(toks) + i + 1
+    assert bench.prefill_pairs(w, idx) == brute
+    # the two full prefill workloads: 4 x 512 retrieved tokens shared by all
+    # heads; 128 sink + 2048 single tokens + 512 window per kv head
+    c2 = W["memlong-cosine-prefill"]
+    idx2 = np.tile(np.arange(4), (c2.n_chunks, 1, 1))
+    assert bench.prefill_pairs(c2, idx2) == 8 * 32 * (512 * 2048 + 512 * 513 // 2)
+    c5 = W["token-retrieval-prefill-1m"]
+    idx5 = np.tile(np.arange(128, 128 + 2048), (1, c5.n_kv_heads, 1))
+    assert bench.prefill_pairs(c5, idx5) == 32 * (2048 * 2688 + 2048 * 2049 // 2)
