@@ -163,15 +163,18 @@ rba_status rba_topk(const float* scores, int32_t rows, int32_t n, int32_t k, int
                     int32_t* idx, void* workspace, size_t ws_bytes, cudaStream_t stream);
 size_t rba_topk_workspace_size(int32_t rows, int32_t n, int32_t k);
 
-/* Decode attention, split-K with online softmax and a log-sum-exp merge of
- * the split partials ([IL] overall framework: local window + a few memory
- * units; [ML] 2.3.3 retrieved chunks attended without a causal mask).
+/* Decode attention with online softmax and a log-sum-exp merge of partial
+ * states ([IL] overall framework: local window + a few memory units; [ML]
+ * 2.3.3 retrieved chunks attended without a causal mask).  Runs the
+ * persistent attention kernel (one CTA per SM, bulk-copy staging) where
+ * rba_decode_step_plan() would report 1, else a split-K kernel.
  *   q    device dtype [B][Hq][D];  idx device int32 [B][Hkv][k] ascending candidate block ids
  *   out  device fp32 [B][Hq][D];   lse device fp32 [B][Hq] (natural log) or NULL
  *   For q head i of kv head h = i / (Hq/Hkv):
  *     out = sum_t softmax_t(scale * q.k_t) v_t over the attended set of (b, h).
- *   workspace >= rba_attend_workspace_size(); its first 4 KiB must be zero before the first
- *   call (the kernels leave it zero after each call that completes).
+ *   workspace >= rba_attend_workspace_size(); its first 2 * roundup256(4 * B * Hkv) bytes
+ *   (merge tickets) must be zero before the first call (the kernels leave them zero after
+ *   each call that completes).
  * Errors: INVALID_ARG (k > nc, T > capacity), WORKSPACE, CUDA; out-of-range idx
  * entries are skipped and flagged as RBA_ERR_BOUNDS in the status word. */
 rba_status rba_attend(const rba_store* store, const void* q, const int32_t* idx, int32_t k,
@@ -186,8 +189,9 @@ size_t rba_attend_workspace_size(const rba_store* store, int32_t k, int64_t T, i
  * Meant for hosts that own all device memory through their own allocator (for
  * example a serving engine that reserves HBM when it starts) and for call sites
  * that cannot afford the device-wide synchronisation cudaMalloc may cause.
- * Same computation, arguments, layouts and errors as rba_attend; the split
- * partials and merge tickets live in a fixed device array inside the library,
+ * Same computation, arguments, layouts and errors as rba_attend, always on the
+ * split-K kernel; its split partials and merge tickets live in a fixed device
+ * array inside the library,
  * RBA_ATTEND_NOALLOC_SCRATCH_BYTES long, which every GPU that loads the library
  * holds until the process exits.
  *   - Allocates nothing: no cudaMalloc / cudaFree and no allocating library call.
@@ -197,8 +201,8 @@ size_t rba_attend_workspace_size(const rba_store* store, int32_t k, int64_t T, i
  *   - Every call shares the one array, which keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other host threads) race and
  *     must be serialised by the caller.
- *   - A call needing more scratch than the limit (see rba_attend_workspace_size)
- *     returns RBA_ERR_WORKSPACE and launches nothing. */
+ *   - A call whose split-K scratch exceeds the limit returns RBA_ERR_WORKSPACE and
+ *     launches nothing. */
 #define RBA_ATTEND_NOALLOC_SCRATCH_BYTES ((size_t)2 << 20)
 rba_status rba_attend_noalloc(const rba_store* store, const void* q, const int32_t* idx,
                               int32_t k, int64_t T, int32_t sink, int32_t window, float scale,
@@ -226,10 +230,15 @@ size_t rba_attend_prefill_workspace_size(const rba_store* store, int32_t n_chunk
                                          int32_t sink, int32_t window);
 
 /* One whole decode step: rba_score (dot modes) -> rba_topk per (b, kv head)
- * -> rba_attend, with the same definitions as those calls.
+ * -> rba_attend, with the same definitions as those calls, as three kernels
+ * on `stream`.  Where rba_decode_step_plan() reports 1, the top-k kernel and
+ * the persistent attention kernel are programmatic dependents of the kernel
+ * before them: they start early, the attention kernel streams the sink and
+ * window rows, and each waits on the device for its inputs.
  *   q device dtype [B][Hq][D]; idx device int32 [B][Hkv][k] (written); scores device fp32
  *   [B][Hkv][nc] (written) or NULL; out/lse as rba_attend.
- *   workspace >= rba_decode_step_workspace_size(); first 4 KiB zero before the first call.
+ *   workspace >= rba_decode_step_workspace_size(); it starts with rba_attend's workspace,
+ *   whose ticket words must be zero before the first call.
  * Errors: as the three calls. */
 rba_status rba_decode_step(const rba_store* store, const void* q, int32_t k, int64_t T,
                            int32_t sink, int32_t window, float scale, float* scores,
@@ -239,11 +248,11 @@ size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t
                                       int32_t sink, int32_t window);
 
 /* How rba_decode_step runs this problem (host only; queries the device, launches nothing):
- *   1   one persistent launch: scores, selection and attention fused; candidates per
- *       (b, kv head) <= 8192, k <= 1024, GQA group of 1, 2 or 4
- *   0   three launches (rba_score, rba_topk, rba_attend): outside those limits
- *  -2   within the limits but no CTA of the fused kernel fits on an SM (three launches)
- *  -3   a CUDA error while asking (three launches)
+ *   1   score -> top-k -> persistent attention kernel, the last two as programmatic
+ *       dependents (overlapped); k <= 2048, GQA group of 1, 2 or 4
+ *   0   score -> top-k -> split-K attention, in stream order: outside those limits
+ *  -2   within the limits but no CTA of the persistent kernel fits on an SM (as 0)
+ *  -3   a CUDA error while asking (as 0)
  *  -4   invalid arguments (as rba_decode_step would report) */
 int32_t rba_decode_step_plan(const rba_store* store, int32_t k, int64_t T, int32_t sink,
                              int32_t window);

@@ -114,6 +114,12 @@ size_t attend_workspace_bytes(int BH, int Hq_total, int D, int nsplit) {
   return attend_layout(nullptr, BH, Hq_total, D, nsplit).bytes;
 }
 
+size_t splitk_workspace_bytes(const rba_store* st, const Geometry& g, int k) {
+  const int BH = st->d.batch * st->d.n_kv_heads;
+  const int nsplit = attend_nsplit(BH, n_att_bound(g, k));
+  return attend_workspace_bytes(BH, st->d.batch * st->d.n_q_heads, st->d.head_dim, nsplit);
+}
+
 rba_status launch_attend(const rba_store* st, const void* q, const int32_t* idx, int k,
                          const Geometry& g, float scale, float* out, float* lse, void* ws,
                          size_t ws_bytes, cudaStream_t stream) {
@@ -156,32 +162,67 @@ rba_status launch_attend(const rba_store* st, const void* q, const int32_t* idx,
 
 namespace {
 
-struct StepWs {
+// Attention workspace: [persistent-kernel tickets (zero)] [split-K tickets
+// (zero) + partials] [persistent-kernel partial slots].  The zero words of
+// the two kernels never overlap the other kernel's scratch.
+struct AttendLayout {
   void* fused_sync;
   float* fused_slots;
-  float* scores;
-  void* topk_ws;
-  size_t topk_bytes;
-  void* attend_ws;
-  size_t attend_bytes;
+  void* splitk_ws;
+  size_t splitk_bytes;
   size_t total;
 };
 
-// [fused sync words (zero)] [attend: tickets (zero) + partials] [scores]
-// [top-k scratch] [fused partial slots]: the zero words of the two paths
-// never overlap the other path's scratch.
-StepWs step_layout(void* ws, const rba_store* st, const Geometry& g, int k, bool own_scores) {
+AttendLayout attend_layout_full(void* ws, const rba_store* st, const Geometry& g, int k) {
   const rba_store_desc& d = st->d;
   const int BH = d.batch * d.n_kv_heads;
-  StepWs s;
+  AttendLayout l;
   char* p = static_cast<char*>(ws);
   size_t off = 0;
-  s.fused_sync = p + off;
+  l.fused_sync = p + off;
   off += fused_sync_bytes(st);
   const int nsplit = attend_nsplit(BH, n_att_bound(g, k));
-  s.attend_bytes = attend_workspace_bytes(BH, d.batch * d.n_q_heads, d.head_dim, nsplit);
-  s.attend_ws = p + off;
-  off += align_up(s.attend_bytes, 256);
+  l.splitk_bytes = attend_workspace_bytes(BH, d.batch * d.n_q_heads, d.head_dim, nsplit);
+  l.splitk_ws = p + off;
+  off += align_up(l.splitk_bytes, 256);
+  l.fused_slots = reinterpret_cast<float*>(p + off);
+  if (fused_eligible(st, g, k)) off += fused_slot_bytes(st, g, k, nullptr);
+  l.total = off;
+  return l;
+}
+
+bool use_fused(const rba_store* st, const Geometry& g, int k) {
+  return fused_eligible(st, g, k) && fused_occupancy(st) > 0;
+}
+
+// Attention over sink U selected blocks U window: the persistent kernel
+// where it applies (pdl: behind the top-k kernel), else split-K.
+rba_status attend_any(const rba_store* st, const void* q, const int32_t* idx, int k,
+                      const Geometry& g, float scale, float* out, float* lse,
+                      const AttendLayout& l, bool pdl, cudaStream_t stream) {
+  if (use_fused(st, g, k)) {
+    const rba_status s =
+        launch_fused(st, q, k, g, scale, idx, out, lse, l.fused_sync, l.fused_slots, pdl, stream);
+    if (s != RBA_ERR_UNSUPPORTED) return s;
+  }
+  return launch_attend(st, q, idx, k, g, scale, out, lse, l.splitk_ws, l.splitk_bytes, stream);
+}
+
+struct StepWs {
+  AttendLayout att;
+  float* scores;
+  void* topk_ws;
+  size_t topk_bytes;
+  size_t total;
+};
+
+// [attention workspace] [scores] [top-k scratch]
+StepWs step_layout(void* ws, const rba_store* st, const Geometry& g, int k, bool own_scores) {
+  const int BH = st->d.batch * st->d.n_kv_heads;
+  StepWs s;
+  char* p = static_cast<char*>(ws);
+  s.att = attend_layout_full(ws, st, g, k);
+  size_t off = align_up(s.att.total, 256);
   s.scores = nullptr;
   if (own_scores) {
     s.scores = reinterpret_cast<float*>(p + off);
@@ -190,8 +231,6 @@ StepWs step_layout(void* ws, const rba_store* st, const Geometry& g, int k, bool
   s.topk_bytes = topk_workspace(BH, g.nc, k);
   s.topk_ws = p + off;
   off += align_up(s.topk_bytes, 256);
-  s.fused_slots = reinterpret_cast<float*>(p + off);
-  off += fused_slot_bytes(st, g, k, nullptr);
   s.total = off;
   return s;
 }
@@ -211,7 +250,9 @@ rba_status rba_attend(const rba_store* st, const void* q, const int32_t* idx, in
   rba_status s = geometry(st, T, sink, window, &g);
   if (s != RBA_OK) return s;
   if (k > g.nc || (k > 0 && idx == nullptr)) return RBA_ERR_INVALID_ARG;
-  return launch_attend(st, q, idx, k, g, scale, out, lse, workspace, ws_bytes, stream);
+  const AttendLayout l = attend_layout_full(workspace, st, g, k);
+  if (workspace == nullptr || ws_bytes < l.total) return RBA_ERR_WORKSPACE;
+  return attend_any(st, q, idx, k, g, scale, out, lse, l, false, stream);
 }
 
 size_t rba_attend_workspace_size(const rba_store* st, int32_t k, int64_t T, int32_t sink,
@@ -219,9 +260,7 @@ size_t rba_attend_workspace_size(const rba_store* st, int32_t k, int64_t T, int3
   using namespace rba;
   Geometry g;
   if (st == nullptr || geometry(st, T, sink, window, &g) != RBA_OK || k < 0) return 0;
-  const int BH = st->d.batch * st->d.n_kv_heads;
-  const int nsplit = attend_nsplit(BH, n_att_bound(g, k));
-  return attend_workspace_bytes(BH, st->d.batch * st->d.n_q_heads, st->d.head_dim, nsplit);
+  return attend_layout_full(nullptr, st, g, k).total;
 }
 
 rba_status rba_decode_step(const rba_store* st, const void* q, int32_t k, int64_t T,
@@ -242,17 +281,17 @@ rba_status rba_decode_step(const rba_store* st, const void* q, int32_t k, int64_
   const int BH = st->d.batch * st->d.n_kv_heads;
   const int grp = st->d.n_q_heads / st->d.n_kv_heads;
   if (grp > 64) return RBA_ERR_UNSUPPORTED;
-  if (fused_eligible(st, g, k)) {
-    s = launch_fused(st, q, k, g, scale, sc, idx, out, lse, w.fused_sync, w.fused_slots, stream);
-    if (s != RBA_ERR_UNSUPPORTED) return s;
-  }
+  // score -> top-k -> attention; the top-k kernel and the persistent
+  // attention kernel start early (programmatic dependent launch) and wait
+  // for their inputs on the device
+  const bool fused = use_fused(st, g, k);
   if (k > 0) {
     s = launch_score_dot(st, q, 1, nullptr, g, sc, stream);
     if (s != RBA_OK) return s;
-    s = launch_topk(sc, BH, g.nc, k, g.first, idx, w.topk_ws, w.topk_bytes, stream);
+    s = launch_topk(sc, BH, g.nc, k, g.first, idx, w.topk_ws, w.topk_bytes, stream, fused);
     if (s != RBA_OK) return s;
   }
-  return launch_attend(st, q, idx, k, g, scale, out, lse, w.attend_ws, w.attend_bytes, stream);
+  return attend_any(st, q, idx, k, g, scale, out, lse, w.att, fused && k > 0, stream);
 }
 
 int32_t rba_decode_step_plan(const rba_store* st, int32_t k, int64_t T, int32_t sink,

@@ -417,6 +417,8 @@ __device__ __forceinline__ void merge_partials_last(const AttendArgs& a, int bh,
 
 // host helpers
 size_t attend_workspace_bytes(int BH, int Hq_total, int D, int nsplit);
+// workspace of the split-K kernel alone for this problem
+size_t splitk_workspace_bytes(const rba_store* st, const Geometry& g, int k);
 int attend_nsplit(int BH, int64_t n_att_max);
 rba_status launch_attend(const rba_store* st, const void* q, const int32_t* idx, int k,
                          const Geometry& g, float scale, float* out, float* lse, void* ws,

@@ -56,7 +56,7 @@ extern "C" rba_status rba_attend_noalloc(const rba_store* st, const void* q, con
   if (s != RBA_OK) return s;
   if (k > g.nc || (k > 0 && idx == nullptr)) return RBA_ERR_INVALID_ARG;
   // reject sizes whose scratch does not fit the fixed array
-  const size_t need = rba_attend_workspace_size(st, k, T, sink, window);
+  const size_t need = splitk_workspace_bytes(st, g, k);
   if (need == 0 || need > kScratchBytes) return RBA_ERR_WORKSPACE;
   void* scratch = nullptr;
   s = scratch_address(&scratch);

@@ -13,19 +13,42 @@
 namespace rba {
 namespace {
 
-// qsum[bh][d] = sum over the group's q heads and n_q rows of q[b][hq][t][d]
-template <typename QT>
-__global__ void qsum_kernel(const QT* __restrict__ q, float* __restrict__ qsum, int Hq, int Hkv,
-                            int n_q, int D) {
+// qsum[bh][d] = sum over the group's q heads and n_q rows of q[b][hq][t][d].
+// The g * n_q rows of one (b, kv head) are contiguous; the CTA reads them as
+// 16-byte vectors (LPR lanes per row, kQsumThreads / LPR rows in flight) and
+// sums the per-thread partials in a fixed order (deterministic).
+constexpr int kQsumThreads = 1024;
+
+template <typename QT, int D>
+__global__ void __launch_bounds__(kQsumThreads) qsum_kernel(const QT* __restrict__ q,
+                                                            float* __restrict__ qsum, int Hq,
+                                                            int Hkv, int n_q) {
+  constexpr int EPV = Elem<QT>::kPerVec;
+  constexpr int LPR = D / EPV;                  // lanes per row
+  constexpr int RPP = kQsumThreads / LPR;       // rows per pass
+  __shared__ float part[RPP][D + 1];
   const int bh = blockIdx.x;
   const int b = bh / Hkv, h = bh % Hkv, g = Hq / Hkv;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < g; ++i) {
-      const QT* base = q + ((int64_t(b) * Hq + h * g + i) * n_q) * D + d;
-      for (int t = 0; t < n_q; ++t) acc += Elem<QT>::to_f32(base[int64_t(t) * D]);
-    }
-    qsum[int64_t(bh) * D + d] = acc;
+  const int64_t rows = int64_t(g) * n_q;
+  const uint4* base = reinterpret_cast<const uint4*>(q + (int64_t(b) * Hq + h * g) * n_q * D);
+  const int sub = threadIdx.x % LPR, r0 = threadIdx.x / LPR;
+  float acc[EPV];
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int64_t r = r0; r < rows; r += RPP) {
+    float f[EPV];
+    unpack(ld_stream(base + r * LPR + sub), f, QT());
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) acc[e] += f[e];
+  }
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) part[r0][sub * EPV + e] = acc[e];
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += kQsumThreads) {
+    float s = 0.f;
+    for (int i = 0; i < RPP; ++i) s += part[i][d];
+    qsum[int64_t(bh) * D + d] = s;
   }
 }
 
@@ -68,13 +91,17 @@ rba_status launch_qsum(const rba_store* st, const void* q, int n_q, float* qsum,
                        cudaStream_t stream) {
   const rba_store_desc& d = st->d;
   const int BH = d.batch * d.n_kv_heads;
-  if (d.dtype == RBA_BF16)
-    qsum_kernel<__nv_bfloat16><<<BH, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(q),
-                                                        qsum, d.n_q_heads, d.n_kv_heads, n_q,
-                                                        d.head_dim);
-  else
-    qsum_kernel<float><<<BH, 128, 0, stream>>>(static_cast<const float*>(q), qsum, d.n_q_heads,
-                                               d.n_kv_heads, n_q, d.head_dim);
+#define RBA_QSUM(QT_, D_)                                                                \
+  qsum_kernel<QT_, D_><<<BH, kQsumThreads, 0, stream>>>(static_cast<const QT_*>(q), qsum, \
+                                                         d.n_q_heads, d.n_kv_heads, n_q)
+  if (d.dtype == RBA_BF16) {
+    if (d.head_dim == 128) RBA_QSUM(__nv_bfloat16, 128);
+    else RBA_QSUM(__nv_bfloat16, 64);
+  } else {
+    if (d.head_dim == 128) RBA_QSUM(float, 128);
+    else RBA_QSUM(float, 64);
+  }
+#undef RBA_QSUM
   RBA_LAUNCH_CHECK();
   return RBA_OK;
 }

@@ -26,6 +26,10 @@ __global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int can
   constexpr int VPL = VPC / LPC;
   constexpr int CPW = 32 / LPC;
   static_assert(VPC % LPC == 0 && 32 % LPC == 0, "rep row must tile the warp");
+  // a kernel launched behind this one as a programmatic dependent (the
+  // top-k of the decode step) may start now; it waits for our completion
+  // before it reads the scores
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float qs[D];
   const int bh = blockIdx.y;
   const int b = bh / a.Hkv, h = bh - b * a.Hkv, g = a.Hq / a.Hkv;

@@ -13,8 +13,10 @@ constexpr int kLargeMaxK = 16384;
 size_t topk_large_workspace(int rows, int n, int k);
 rba_status launch_topk_large(const float* scores, int rows, int n, int k, int index_base,
                              int32_t* idx, void* ws, cudaStream_t stream);
+// pdl: launched as a programmatic dependent of the previous kernel on the
+// stream (it waits for that kernel's completion before reading scores)
 rba_status launch_topk(const float* scores, int rows, int n, int k, int index_base, int32_t* idx,
-                       void* ws, size_t ws_bytes, cudaStream_t stream);
+                       void* ws, size_t ws_bytes, cudaStream_t stream, bool pdl);
 size_t topk_workspace(int rows, int n, int k);
 
 }  // namespace rba

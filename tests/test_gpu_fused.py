@@ -1,9 +1,11 @@
-"""The whole decode step in one launch (rba_decode_step) against the
-three-launch path (rba_score -> rba_topk -> rba_attend) on the same store:
-identical selections, outputs within the attention tolerance.  Shapes cover
-one CTA per SM, grids smaller than the SM count, several heads per CTA, GQA
-groups of 1, 2 and 4, ragged block sizes, and repeated calls on one
-workspace (its synchronisation words must come back to zero)."""
+"""The whole decode step (rba_decode_step: score, top-k and the persistent
+attention kernel, the last two launched as programmatic dependents that start
+early and wait on the device) against the same three calls made one after the
+other (rba_score -> rba_topk -> rba_attend) on the same store: identical
+selections, outputs within the attention tolerance.  Shapes cover one CTA per
+SM, grids smaller than the SM count, several heads per CTA, GQA groups of 1, 2
+and 4, ragged block sizes, and repeated calls on one workspace (its merge
+tickets must come back to zero)."""
 import numpy as np
 import pytest
 import torch

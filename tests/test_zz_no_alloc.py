@@ -71,3 +71,45 @@ def test_noalloc_rejects_sizes_beyond_the_limit(rba):
     out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device="cuda")
     lse = torch.empty((w.batch, w.n_q_heads), device="cuda")
     assert _noalloc(rba, st, q, idx, w, out, lse) == rba.ERR_WORKSPACE
+
+
+SPLIT_K_CASES = {
+    "tiny-decode-f32": synth.WORKLOADS["tiny-decode-f32"],
+    "ragged-f32": synth.WORKLOADS["tiny-decode-f32"].scaled(
+        n_q_heads=8, n_kv_heads=4, context=1000, block_size=24, sink=30, window=70, top_k=7,
+        seed=11),
+    "landmark-small": synth.WORKLOADS["landmark-decode-b16"].scaled(
+        batch=2, n_q_heads=4, n_kv_heads=4, context=5018),
+    "token-small": synth.WORKLOADS["token-retrieval-decode-1m"].scaled(context=65536,
+                                                                         top_k=256),
+}
+
+
+@pytest.mark.parametrize("name", list(SPLIT_K_CASES))
+def test_noalloc_split_k_matches_oracle(rba, name):
+    # rba_attend_noalloc always runs the split-K kernel (rba_attend takes the
+    # persistent kernel where it applies): this is that kernel's parity
+    # against the oracle, on the oracle's own selection
+    from parity import attended_v_max, out_error
+    w = SPLIT_K_CASES[name]
+    x = synth.decode_inputs(w)
+    reps, _ = oracle_reps(w, x)
+    st = make_decode_store(rba, w, x)
+    ref = O.decode(x["q"], x["K"], x["V"], reps, dtype=w.dtype, block_size=w.block_size,
+                   sink=w.sink, window=w.window, top_k_blocks=w.top_k)
+    idx = torch.from_numpy(ref["idx"].astype(np.int32)).cuda()
+    q = dev(x["q"], w.dtype)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device="cuda")
+    lse = torch.empty((w.batch, w.n_q_heads), device="cuda")
+    assert _noalloc(rba, st, q, idx, w, out, lse) == rba.OK
+    st.check()
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    g = w.n_q_heads // w.n_kv_heads
+    worst = 0.0
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            va = attended_v_max(w, x, b, h, ref["idx"][b, h])
+            for i in range(h * g, (h + 1) * g):
+                worst = max(worst, out_error(out[b, i], ref["out"][b, i], va))
+    assert worst <= OUT_TOL[w.dtype], worst
+    np.testing.assert_allclose(lse, ref["lse"], rtol=0, atol=OUT_TOL[w.dtype])
