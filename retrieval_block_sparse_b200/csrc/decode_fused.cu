@@ -37,7 +37,6 @@ constexpr int kCT = kCW * 32;                 // compute threads
 constexpr int kFT = kCT + 32;                 // + warp 0, which stages
 constexpr int kMaxK = 2048;                   // selected blocks per (b, kv head)
 constexpr int kMaxStages = 6;
-constexpr int kMaxSlots = 128;                // partial slots per head
 constexpr int kMinRowsPerCta = 128;           // grid shrinks for small problems
 constexpr int kMaxGrid = 256;                 // CTAs (one per SM)
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
@@ -46,9 +45,10 @@ struct FusedArgs {
   AttendArgs at;            // K, V, q, out, lse, status, cap, T, w0, Hq, Hkv, k, bs, sink,
                             // sink_end, first, nc, scale_log2 (part/tickets/nsplit unused)
   int32_t* idx;             // [BH][k], written by the top-k kernel before this one
-  float* slots;             // [BH][MS][G][D+2] partial states, one per contributing CTA
+  float* slots;             // [BH][m][G][D+2] partial states, one per part of a head
   uint32_t* tickets;        // [BH], zero between calls
-  int BH, L_st, U_sel, MS, NS;
+  int BH, L_st, U_sel, NS;
+  int m;                    // parts per head (CTAs per head when BH <= CTAs, else 1)
 };
 
 // ---------------------------------------------------------------------------
@@ -137,36 +137,16 @@ __device__ __forceinline__ int ctid() { return static_cast<int>(threadIdx.x) - 3
 
 // ---------------------------------------------------------------------------
 // work list
-
-__device__ __forceinline__ int64_t bnd(int p, int P, int64_t total) {
-  return total * p / P;
-}
-
-// CTAs whose share of the attention list meets head bh's rows: how many (=
-// the partials that head receives) and the ordinal of CTA `me` among them
-// (its slot), or -1 if it is not one of them.  `B` holds the CTA boundaries
-// bnd(0..P) (no division here).
-__device__ __forceinline__ int contributors(int bh, int64_t per_bh, int P, const int64_t* B,
-                                            int me, int* ordinal) {
-  *ordinal = -1;
-  if (per_bh <= 0) return 0;
-  const int64_t a = bh * per_bh, b = a + per_bh;
-  // first CTA whose range ends after a: the largest p with B[p] <= a
-  int lo = 0, hi = P - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (B[mid] <= a) lo = mid; else hi = mid - 1;
-  }
-  int c = 0;
-  for (int p = lo; p < P && B[p] < b; ++p) {
-    const int64_t s = max(B[p], a), e = min(B[p + 1], b);
-    if (e > s) {
-      if (p == me) *ordinal = c;
-      ++c;
-    }
-  }
-  return c;
-}
+//
+// The attention rows of head h (Lh = L_st + U_sel) are cut into m equal
+// parts, "units" u = h * m + c, c < m; CTA p takes units
+// [U * p / P, U * (p + 1) / P) of the U = BH * m units.  With BH <= P, m is
+// chosen so that P = BH * m: every CTA holds exactly one part of one head and
+// each head has exactly m partial states.  With BH > P, m = 1: every CTA holds
+// whole heads and writes their outputs itself.  A part [x0, x1) of a head
+// maps to sink/window rows [st(x0), st(x1)) and selected rows
+// [x0 - st(x0), x1 - st(x1)) with st(x) = floor(x * L_st / Lh), so a CTA
+// streams both kinds of one head with one softmax state, sink/window first.
 
 struct Item {
   int kind;  // 1 sink/window rows, 2 selected rows
@@ -174,21 +154,18 @@ struct Item {
   int v0, v1;
 };
 
-// A CTA's walk over its share [r, r1) of the flattened attention list, where
-// head h contributes Lh = L_st + U_sel rows.  A share [x0, x1) of head h maps
-// to sink/window rows [st(x0), st(x1)) and selected rows
-// [x0 - st(x0), x1 - st(x1)) with st(x) = floor(x * L_st / Lh), so a CTA
-// streams both parts of one head with one softmax state, sink/window first.
 struct Iter {
-  int64_t r, r1;
-  int bh, kind, v, vend, sel0, sel1;
+  int64_t u, u1;          // current unit, end of this CTA's units
+  int bh, part;           // head and part index of unit u
+  int kind, v, vend, sel0, sel1;
   bool done;
 };
 
-__device__ __forceinline__ void attn_head(const FusedArgs& a, Iter& it) {
-  const int64_t Lh = a.L_st + a.U_sel;
-  const int64_t h0 = int64_t(it.bh) * Lh;
-  const int64_t x0 = max(it.r, h0) - h0, x1 = min(it.r1, h0 + Lh) - h0;
+__device__ __forceinline__ void unit_begin(const FusedArgs& a, Iter& it) {
+  const int64_t Lh = int64_t(a.L_st) + a.U_sel;
+  it.bh = static_cast<int>(it.u / a.m);
+  it.part = static_cast<int>(it.u - int64_t(it.bh) * a.m);
+  const int64_t x0 = Lh * it.part / a.m, x1 = Lh * (it.part + 1) / a.m;
   const int64_t s0 = x0 * a.L_st / Lh, s1 = x1 * a.L_st / Lh;
   it.kind = 1;
   it.v = static_cast<int>(s0);
@@ -197,15 +174,12 @@ __device__ __forceinline__ void attn_head(const FusedArgs& a, Iter& it) {
   it.sel1 = static_cast<int>(x1 - s1);
 }
 
-// B: CTA boundaries of the attention list
-__device__ __forceinline__ void iter_begin(const FusedArgs& a, Iter& it, const int64_t* B) {
-  it.r = B[blockIdx.x];
-  it.r1 = B[blockIdx.x + 1];
-  it.done = it.r >= it.r1;
-  if (!it.done) {
-    it.bh = static_cast<int>(it.r / (int64_t(a.L_st) + a.U_sel));
-    attn_head(a, it);
-  }
+__device__ __forceinline__ void iter_begin(const FusedArgs& a, Iter& it) {
+  const int64_t U = int64_t(a.BH) * a.m;
+  it.u = U * blockIdx.x / gridDim.x;
+  it.u1 = U * (blockIdx.x + 1) / gridDim.x;
+  it.done = it.u >= it.u1;
+  if (!it.done) unit_begin(a, it);
 }
 
 template <int TT>
@@ -226,12 +200,11 @@ __device__ __forceinline__ bool next_item(const FusedArgs& a, Iter& it, Item& ou
       it.vend = it.sel1;
       continue;
     }
-    ++it.bh;
-    if (int64_t(it.bh) * (int64_t(a.L_st) + a.U_sel) >= it.r1) {
+    if (++it.u >= it.u1) {
       it.done = true;
       break;
     }
-    attn_head(a, it);
+    unit_begin(a, it);
   }
   return false;
 }
@@ -252,10 +225,8 @@ struct FusedSmem {
   // regions after the stage ring (NS * STAGE, chosen at launch)
   static constexpr int RED = up16(kCW * G * (D + 2) * 4);       // warp states / merge sums
   static constexpr int SEL = (kMaxK + 4) * 4 * 2;               // selected prefix + starts
-  static constexpr int SLOTS = up16((3 * G * kMaxSlots) * 4);   // merge: m, l, w
   static constexpr int MISC = 1024;
-  static constexpr int BOUNDS = (kMaxGrid + 1) * 8;             // CTA boundaries
-  static size_t bytes(int NS) { return size_t(NS) * STAGE + RED + SEL + SLOTS + MISC + BOUNDS; }
+  static size_t bytes(int NS) { return size_t(NS) * STAGE + RED + SEL + MISC; }
 };
 
 // LaneState query slice from a [G][D] fp32 copy in shared memory (the same
@@ -380,12 +351,11 @@ __device__ void issue_item(const FusedArgs& a, const Item& item, char* stg, uint
 template <typename T, int D>
 __device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64_t* full,
                                         uint64_t* empty, Meta* meta, int* sel_pref,
-                                        int* sel_phys, volatile int* abort_flag,
-                                        const int64_t* B) {
+                                        int* sel_phys, volatile int* abort_flag) {
   using C = DecodeTile<T, D, kCW>;
   const int NS = a.NS;
   Iter it;
-  iter_begin(a, it, B);
+  iter_begin(a, it);
   Item item;
   int j = 0, s = 0, sel_bh = -1;
   uint32_t ph = 0;  // phase parity of the stage's next fill
@@ -426,19 +396,15 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   float* red = reinterpret_cast<float*>(smem + size_t(NS) * C::STAGE);
   int* sel_pref = reinterpret_cast<int*>(reinterpret_cast<char*>(red) + S::RED);
   int* sel_phys = sel_pref + (kMaxK + 1);
-  float* wslot = reinterpret_cast<float*>(reinterpret_cast<char*>(sel_pref) + S::SEL);
-  char* misc = reinterpret_cast<char*>(wslot) + S::SLOTS;
+  char* misc = reinterpret_cast<char*>(sel_pref) + S::SEL;
   uint64_t* full = reinterpret_cast<uint64_t*>(misc);               // [kMaxStages]
   uint64_t* empty = full + kMaxStages;                              // [kMaxStages]
   Meta* meta = reinterpret_cast<Meta*>(empty + kMaxStages);         // [kMaxStages]
   int* s_misc = reinterpret_cast<int*>(meta + kMaxStages);          // [16]
   volatile int* abort_flag = s_misc + 16;                           // [4]
   float* s_f = reinterpret_cast<float*>(s_misc + 20);               // [32]
-  int64_t* B = reinterpret_cast<int64_t*>(misc + S::MISC);          // [P+1]
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int P = gridDim.x, p = blockIdx.x;
-  const int64_t Lh = int64_t(a.L_st) + a.U_sel;
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
@@ -448,10 +414,9 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  for (int q = threadIdx.x; q <= P; q += kFT) B[q] = bnd(q, P, Lh * a.BH);
   __syncthreads();
   if (warp == 0) {
-    produce<T, D>(a, stages, full, empty, meta, sel_pref, sel_phys, abort_flag, B);
+    produce<T, D>(a, stages, full, empty, meta, sel_pref, sel_phys, abort_flag);
     return;
   }
   // ---- compute warps from here on (named barrier 1; no __syncthreads)
@@ -473,7 +438,9 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   };
 
   // the query heads of this CTA's first head, fp32, while the first tile loads
-  const int bh_att0 = B[p] < B[p + 1] ? static_cast<int>(B[p] / Lh) : -1;
+  Iter it;
+  iter_begin(a, it);
+  const int bh_att0 = it.done ? -1 : it.bh;
   float* q_first = red;  // [G][D]; red is not used before the first flush
   if (bh_att0 >= 0) {
     const int b = bh_att0 / a.at.Hkv, h = bh_att0 % a.at.Hkv;
@@ -482,17 +449,13 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   }
   compute_sync();
 
-  Iter it;
-  iter_begin(a, it, B);
   Item item;
   bool have = next_item<C::TT>(a, it, item);
 
   // ---- attention over this CTA's rows, head by head
   LaneState<T, D, G> st;
   int cur_bh = -1;
-  float* m_s = wslot;                           // [nl][G]
-  float* l_s = m_s + G * kMaxSlots;             // [nl][G]
-  float* w_s = l_s + G * kMaxSlots;             // [G][nl]
+  int ord = 0;  // part index of head cur_bh held by this CTA (its slot)
   while (true) {
     const bool more = have;
     if (cur_bh >= 0 && (!more || item.bh != cur_bh)) {
@@ -525,105 +488,140 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
       // per q head: the CTA's max over warps and each warp's factor exp2(m_w - M)
       float* fac = s_f;         // [G][kCW]
       float* gmax = s_f + 28;   // [G]
-      if (tid < G) {
+      if (tid < G * kCW) {
+        const int gg = tid / kCW, w = tid % kCW;
         float M = -INFINITY;
-        for (int w = 0; w < kCW; ++w) M = fmaxf(M, red[(w * G + tid) * (D + 2)]);
-        for (int w = 0; w < kCW; ++w) {
-          const float mw = red[(w * G + tid) * (D + 2)];
-          fac[tid * kCW + w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
-        }
-        gmax[tid] = M;
-      }
-      int ord;
-      const int ncontrib = contributors(cur_bh, Lh, P, B, p, &ord);
-      const bool slot_ok = ord >= 0 && ord < a.MS;
-      if (!slot_ok && tid == 0) report(a.at.status, RBA_ERR_BOUNDS, kWhereFused, 4);
-      float* base = a.slots + int64_t(cur_bh) * a.MS * G * (D + 2);
-      float* slot = base + int64_t(slot_ok ? ord : 0) * G * (D + 2);
-      compute_sync();
-#pragma unroll 1
-      for (int x = tid; x < G * (D + 2) && slot_ok; x += kCT) {
-        const int gg = x / (D + 2), c = x % (D + 2);
-        float acc = 0.f;
-        if (c == 0) {
-          acc = gmax[gg];
-        } else {
 #pragma unroll
-          for (int w = 0; w < kCW; ++w) acc += red[(w * G + gg) * (D + 2) + c] * fac[gg * kCW + w];
-        }
-        slot[x] = acc;
+        for (int v = 0; v < kCW; ++v) M = fmaxf(M, red[(v * G + gg) * (D + 2)]);
+        const float mw = red[(w * G + gg) * (D + 2)];
+        fac[tid] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+        if (w == 0) gmax[gg] = M;
       }
       compute_sync();
-      if (tid == 0) {
-        const uint32_t t = atom_add_acq_rel(a.tickets + cur_bh, 1u);  // publishes our slot
-        s_misc[9] = t == uint32_t(ncontrib - 1);
-      }
-      compute_sync();
-      if (s_misc[9]) {
-        const int nl = min(ncontrib, a.MS);
-        for (int x = tid; x < nl * G; x += kCT) {  // (m, l) of every slot, one round trip
-          const int j = x / G, gg = x % G;
-          const float* sp = base + (int64_t(j) * G + gg) * (D + 2);
-          m_s[x] = __ldcg(sp);
-          l_s[x] = __ldcg(sp + 1);
-        }
-        compute_sync();
-        if (cw < G) {
-          const int gg = cw;
-          float M = -INFINITY;
-          for (int j = lane; j < nl; j += 32) M = fmaxf(M, m_s[j * G + gg]);
-          for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-          float L = 0.f;
-          for (int j = lane; j < nl; j += 32) {
-            const float ms_ = m_s[j * G + gg];
-            const float wv = ms_ == -INFINITY ? 0.f : exp2f(ms_ - M);
-            w_s[gg * kMaxSlots + j] = wv;
-            L += wv * l_s[j * G + gg];
+      // output of head cur_bh from the warp states in red, combined with fac
+      auto write_out = [&]() {
+        const int b = cur_bh / a.at.Hkv, h = cur_bh % a.at.Hkv;
+        for (int x = tid; x < G * D; x += kCT) {
+          const int gg = x / D, d = x % D;
+          float num = 0.f, den = 0.f;
+#pragma unroll
+          for (int w = 0; w < kCW; ++w) {
+            const float f = fac[gg * kCW + w];
+            num += red[(w * G + gg) * (D + 2) + 2 + d] * f;
+            den += red[(w * G + gg) * (D + 2) + 1] * f;
           }
-          for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          for (int j = lane; j < nl; j += 32) w_s[gg * kMaxSlots + j] *= inv;
-          if (lane == 0 && a.at.lse != nullptr) {
-            const int b = cur_bh / a.at.Hkv, h = cur_bh % a.at.Hkv;
+          a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = den > 0.f ? num / den : 0.f;
+          if (d == 0 && a.at.lse != nullptr)
             a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
-                L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+                den > 0.f ? (gmax[gg] + log2f(den)) * 0.6931471805599453f : -INFINITY;
+        }
+      };
+      if (a.m == 1) {
+        write_out();  // this CTA holds the whole head
+      } else {
+        // this CTA's state -> slot `ord` of the head; the last of the head's
+        // m parts to finish merges all m slots
+        const bool slot_ok = ord >= 0 && ord < a.m;
+        if (!slot_ok && tid == 0) report(a.at.status, RBA_ERR_BOUNDS, kWhereFused, 4);
+        float* base = a.slots + int64_t(cur_bh) * a.m * G * (D + 2);
+        float* slot = base + int64_t(slot_ok ? ord : 0) * G * (D + 2);
+#pragma unroll 1
+        for (int x = tid; x < G * (D + 2) && slot_ok; x += kCT) {
+          const int gg = x / (D + 2), c = x % (D + 2);
+          float acc = 0.f;
+          if (c == 0) {
+            acc = gmax[gg];
+          } else {
+#pragma unroll
+            for (int w = 0; w < kCW; ++w)
+              acc += red[(w * G + gg) * (D + 2) + c] * fac[gg * kCW + w];
           }
+          slot[x] = acc;
         }
         compute_sync();
-        // warps take slots round-robin and read each slot whole (coalesced)
-        constexpr int PER = (G * D + 31) / 32;
-        float acc[PER];
+        if (tid == 0) {
+          const uint32_t t = atom_add_acq_rel(a.tickets + cur_bh, 1u);  // publishes our slot
+          s_misc[9] = t == uint32_t(a.m - 1);
+        }
+        compute_sync();
+        if (s_misc[9]) {
+          // each warp folds whole slots j = cw, cw + kCW, ... into a running
+          // (max, sum, output) per q head, three slots' loads in flight at
+          // once; then the warps' states are combined through red
+          const int nl = a.m;
+          constexpr int PER = (G * D + 31) / 32;  // output elements (g, d) per lane
+          constexpr int UN = 2;
+          float O[PER], M[G], L[G];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+          for (int e = 0; e < PER; ++e) O[e] = 0.f;
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg) {
+            M[gg] = -INFINITY;
+            L[gg] = 0.f;
+          }
 #pragma unroll 1
-        for (int j = cw; j < nl; j += kCW) {
-          const float* sp = base + int64_t(j) * G * (D + 2);
-          float v[PER];
+          for (int j0 = cw; j0 < nl; j0 += UN * kCW) {
+            float v[UN][PER], mj[UN][G], lj[UN][G];
 #pragma unroll
-          for (int e = 0; e < PER; ++e) {
-            const int x = lane + 32 * e;  // output element (g, d)
-            v[e] = x < G * D ? __ldcg(sp + (x / D) * (D + 2) + 2 + (x % D)) : 0.f;
+            for (int u = 0; u < UN; ++u) {
+              const int j = j0 + u * kCW;
+              const float* sp = base + int64_t(j < nl ? j : 0) * G * (D + 2);
+#pragma unroll
+              for (int gg = 0; gg < G; ++gg) {
+                mj[u][gg] = j < nl ? __ldcg(sp + gg * (D + 2)) : -INFINITY;
+                lj[u][gg] = j < nl ? __ldcg(sp + gg * (D + 2) + 1) : 0.f;
+              }
+#pragma unroll
+              for (int e = 0; e < PER; ++e) {
+                const int x = lane + 32 * e;
+                v[u][e] = j < nl && x < G * D ? __ldcg(sp + (x / D) * (D + 2) + 2 + (x % D))
+                                              : 0.f;
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < UN; ++u) {
+              float sa[G], sb[G];
+#pragma unroll
+              for (int gg = 0; gg < G; ++gg) {
+                const float mn = fmaxf(M[gg], mj[u][gg]);
+                sa[gg] = M[gg] == -INFINITY ? 0.f : exp2f(M[gg] - mn);
+                sb[gg] = mj[u][gg] == -INFINITY ? 0.f : exp2f(mj[u][gg] - mn);
+                L[gg] = L[gg] * sa[gg] + lj[u][gg] * sb[gg];
+                M[gg] = mn;
+              }
+#pragma unroll
+              for (int e = 0; e < PER; ++e) {
+                const int gg = (lane + 32 * e) / D;
+                if (gg < G) O[e] = O[e] * sa[gg] + v[u][e] * sb[gg];
+              }
+            }
           }
 #pragma unroll
           for (int e = 0; e < PER; ++e) {
             const int x = lane + 32 * e;
-            if (x < G * D) acc[e] += w_s[(x / D) * kMaxSlots + j] * v[e];
+            if (x < G * D) red[(cw * G + x / D) * (D + 2) + 2 + x % D] = O[e];
           }
-        }
+          if (lane == 0) {
 #pragma unroll
-        for (int e = 0; e < PER; ++e) {
-          const int x = lane + 32 * e;
-          if (x < G * D) red[cw * G * D + x] = acc[e];
+            for (int gg = 0; gg < G; ++gg) {
+              red[(cw * G + gg) * (D + 2)] = M[gg];
+              red[(cw * G + gg) * (D + 2) + 1] = L[gg];
+            }
+          }
+          compute_sync();
+          if (tid < G * kCW) {
+            const int gg = tid / kCW, w = tid % kCW;
+            float Mx = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < kCW; ++q) Mx = fmaxf(Mx, red[(q * G + gg) * (D + 2)]);
+            const float mw = red[(w * G + gg) * (D + 2)];
+            fac[tid] = mw == -INFINITY ? 0.f : exp2f(mw - Mx);
+            if (w == 0) gmax[gg] = Mx;
+          }
+          compute_sync();
+          write_out();
+          if (tid == 0) a.tickets[cur_bh] = 0;  // zero again for the next call
         }
-        compute_sync();
-        for (int x = tid; x < G * D; x += kCT) {
-          float sum = 0.f;
-          for (int w = 0; w < kCW; ++w) sum += red[w * G * D + x];
-          const int gg = x / D, d = x % D;
-          const int b = cur_bh / a.at.Hkv, h = cur_bh % a.at.Hkv;
-          a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = sum;
-        }
-        if (tid == 0) a.tickets[cur_bh] = 0;  // zero again for the next call
       }
       compute_sync();
       cur_bh = -1;
@@ -635,6 +633,7 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
         load_q_smem<T, D, G>(q_first, a.at.scale_log2, st);
       else
         load_q<T, D, G>(a.at, cur_bh, st);
+      ord = it.part;
     }
     if (wait_full()) {
       consume_tile<T, D, G, kCW>(stages + size_t(s) * C::STAGE, meta[s].nrows, st, cw);
@@ -709,10 +708,10 @@ static int64_t attention_rows(const rba_store* st, const Geometry& g, int k) {
   return BH * (int64_t(g.sink_end) + (g.T - g.w0) + (k > 0 ? int64_t(k) * st->d.block_size : 0));
 }
 
-// CTAs of the attention launch: one per SM, leaving the SMs that the top-k
-// kernel (one CTA per row) holds while this kernel starts; fewer for small
-// problems.
-int fused_grid(const rba_store* st, const Geometry& g, int k) {
+// CTAs available to the attention launch: one per SM, leaving the SMs that
+// the top-k kernel (one CTA per row) holds while this kernel starts; fewer
+// for small problems.
+static int cta_budget(const rba_store* st, const Geometry& g, int k) {
   const int BH = st->d.batch * st->d.n_kv_heads;
   int sms = num_sms();
   if (k > 0 && g.nc <= kSmallN && BH <= sms / 4) sms -= BH;
@@ -722,27 +721,35 @@ int fused_grid(const rba_store* st, const Geometry& g, int k) {
   return static_cast<int>(P < 1 ? 1 : P);
 }
 
-// Bound on the CTAs whose share of the attention list meets one head's rows
-// (each contributor holds at least one of the head's rows, and at least
-// floor(total / P) rows in all).
-static int slots_bound(int64_t per_bh, int64_t total, int P) {
-  if (per_bh <= 0) return 0;
-  int64_t minlen = total / P;
-  if (minlen < 1) minlen = 1;
-  int64_t b = (per_bh + minlen - 1) / minlen + 1;
-  if (b > per_bh) b = per_bh;
-  return static_cast<int>(b);
+// Parts per head (m) and CTAs (P): with BH <= budget, m = budget / BH and
+// P = BH * m (each CTA one part of one head); else m = 1 and P = budget
+// (each CTA whole heads).
+static void partition(const rba_store* st, const Geometry& g, int k, int* m, int* P) {
+  const int BH = st->d.batch * st->d.n_kv_heads;
+  const int budget = cta_budget(st, g, k);
+  if (BH <= budget) {
+    *m = budget / BH;
+    *P = BH * *m;
+  } else {
+    *m = 1;
+    *P = budget;
+  }
+}
+
+int fused_grid(const rba_store* st, const Geometry& g, int k) {
+  int m, P;
+  partition(st, g, k, &m, &P);
+  return P;
 }
 
 size_t fused_slot_bytes(const rba_store* st, const Geometry& g, int k, int* ms) {
   const rba_store_desc& d = st->d;
   const int BH = d.batch * d.n_kv_heads;
   const int G = d.n_q_heads / d.n_kv_heads;
-  const int P = fused_grid(st, g, k);
-  const int64_t total = attention_rows(st, g, k);
-  const int m = slots_bound(total / BH, total, P);
+  int m, P;
+  partition(st, g, k, &m, &P);
   if (ms) *ms = m;
-  return align_up(size_t(BH) * m * G * (d.head_dim + 2) * 4, 256);
+  return m > 1 ? align_up(size_t(BH) * m * G * (d.head_dim + 2) * 4, 256) : 0;
 }
 
 size_t fused_sync_bytes(const rba_store* st) {
@@ -760,7 +767,7 @@ bool fused_eligible(const rba_store* st, const Geometry& g, int k) {
   if (attention_rows(st, g, k) == 0) return false;
   int ms = 0;
   fused_slot_bytes(st, g, k, &ms);
-  return ms <= kMaxSlots;
+  return ms <= kMaxGrid;
 }
 
 int fused_occupancy(const rba_store* st) {
@@ -816,7 +823,7 @@ rba_status launch_fused(const rba_store* st, const void* q, int k, const Geometr
   a.BH = BH;
   a.L_st = static_cast<int>(g.sink_end + (g.T - g.w0));
   a.U_sel = k > 0 ? k * d.block_size : 0;
-  fused_slot_bytes(st, g, k, &a.MS);
+  fused_slot_bytes(st, g, k, &a.m);
   const int G = d.n_q_heads / d.n_kv_heads;
 #define RBA_FUSED(T_, D_)                                               \
   switch (G) {                                                          \
