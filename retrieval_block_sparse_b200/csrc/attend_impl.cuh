@@ -176,17 +176,21 @@ __device__ __forceinline__ int lane_rot(int part) {
   return (part * C::CPL) / 8;
 }
 
+// Query heads g0 .. g0 + G - 1 of the group of (b, kv head) bh (the group
+// has Hq / Hkv heads).
 template <typename T, int D, int G>
-__device__ __forceinline__ void load_q(const AttendArgs& a, int bh, LaneState<T, D, G>& st) {
+__device__ __forceinline__ void load_q(const AttendArgs& a, int bh, LaneState<T, D, G>& st,
+                                       int g0 = 0) {
   using C = DecodeTile<T, D>;
   const int lane = threadIdx.x & 31;
   const int part = lane % C::LPR;
   const int rot = lane_rot<T, D>(part);
   const int b = bh / a.Hkv, h = bh % a.Hkv;
+  const int grp = a.Hq / a.Hkv;
   const T* q = static_cast<const T*>(a.q);
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const T* qr = q + (int64_t(b) * a.Hq + h * G + g) * D + part * C::EPL;
+    const T* qr = q + (int64_t(b) * a.Hq + h * grp + g0 + g) * D + part * C::EPL;
 #pragma unroll
     for (int j = 0; j < C::CPL; ++j) {
       const int jj = (j + rot) % C::CPL;

@@ -32,23 +32,43 @@
 namespace rba {
 namespace {
 
-constexpr int kCW = 7;                        // compute warps (warps 1..7)
+constexpr int kCW = 14;                       // compute warps (warps 1..14)
 constexpr int kCT = kCW * 32;                 // compute threads
 constexpr int kFT = kCT + 32;                 // + warp 0, which stages
+
+// The compute warps form NGRP groups of RW warps.  With G >= 2 q heads per kv
+// head each group holds HS = G / 2 of them for every row of a tile (the tile
+// is read by both groups; each lane keeps half the softmax state, so 15 warps
+// fit the register file); with G = 1 one group of kCW warps splits the rows.
+template <int G>
+struct Groups {
+  static constexpr int NGRP = G >= 2 ? 2 : 1;
+  static constexpr int HS = G / NGRP;        // q heads per warp
+  static constexpr int RW = kCW / NGRP;      // warps per group (rows of a tile)
+  static_assert(G % NGRP == 0 && kCW % NGRP == 0, "even split");
+};
 constexpr int kMaxK = 2048;                   // selected blocks per (b, kv head)
 constexpr int kMaxStages = 6;
 constexpr int kMinRowsPerCta = 128;           // grid shrinks for small problems
 constexpr int kMaxGrid = 256;                 // CTAs (one per SM)
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
+// One partial state (G q heads x (m, l, o[D]) floats), padded to 16 bytes so
+// that every slot can be moved by a bulk copy.
+__host__ __device__ constexpr int slot_floats(int G, int D) { return (G * (D + 2) + 3) & ~3; }
+
 struct FusedArgs {
   AttendArgs at;            // K, V, q, out, lse, status, cap, T, w0, Hq, Hkv, k, bs, sink,
                             // sink_end, first, nc, scale_log2 (part/tickets/nsplit unused)
   int32_t* idx;             // [BH][k], written by the top-k kernel before this one
-  float* slots;             // [BH][m][G][D+2] partial states, one per part of a head
+  float* slots;             // [BH][m] partial states of slot_floats(G, D), one per part
   uint32_t* tickets;        // [BH], zero between calls
   int BH, L_st, U_sel, NS;
   int m;                    // parts per head (CTAs per head when BH <= CTAs, else 1)
+  // part c of a head: attention rows [px[c], px[c+1]), of which sink/window
+  // rows [ps[c], ps[c+1]) and selected rows [px[c] - ps[c], px[c+1] - ps[c+1])
+  int px[kMaxGrid + 1];
+  int ps[kMaxGrid + 1];
 };
 
 // ---------------------------------------------------------------------------
@@ -75,13 +95,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b))
                : "memory");
 }
+// Tests the phase; a thread whose phase is not complete is suspended until it
+// completes or about 20 us pass (the hint), so waiting warps do not spin.
 __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
+      : "r"(smem_u32(b)), "r"(parity), "r"(20000u)
       : "memory");
   return ok != 0;
 }
@@ -155,29 +177,28 @@ struct Item {
 };
 
 struct Iter {
-  int64_t u, u1;          // current unit, end of this CTA's units
+  int u, u1;              // current unit, end of this CTA's units
   int bh, part;           // head and part index of unit u
   int kind, v, vend, sel0, sel1;
   bool done;
 };
 
 __device__ __forceinline__ void unit_begin(const FusedArgs& a, Iter& it) {
-  const int64_t Lh = int64_t(a.L_st) + a.U_sel;
-  it.bh = static_cast<int>(it.u / a.m);
-  it.part = static_cast<int>(it.u - int64_t(it.bh) * a.m);
-  const int64_t x0 = Lh * it.part / a.m, x1 = Lh * (it.part + 1) / a.m;
-  const int64_t s0 = x0 * a.L_st / Lh, s1 = x1 * a.L_st / Lh;
+  it.bh = it.u / a.m;
+  it.part = it.u - it.bh * a.m;
+  const int x0 = a.px[it.part], x1 = a.px[it.part + 1];
+  const int s0 = a.ps[it.part], s1 = a.ps[it.part + 1];
   it.kind = 1;
-  it.v = static_cast<int>(s0);
-  it.vend = static_cast<int>(s1);
-  it.sel0 = static_cast<int>(x0 - s0);
-  it.sel1 = static_cast<int>(x1 - s1);
+  it.v = s0;
+  it.vend = s1;
+  it.sel0 = x0 - s0;
+  it.sel1 = x1 - s1;
 }
 
 __device__ __forceinline__ void iter_begin(const FusedArgs& a, Iter& it) {
-  const int64_t U = int64_t(a.BH) * a.m;
-  it.u = U * blockIdx.x / gridDim.x;
-  it.u1 = U * (blockIdx.x + 1) / gridDim.x;
+  const unsigned U = unsigned(a.BH) * a.m;  // < 2^24 (host-checked): no overflow below
+  it.u = static_cast<int>(U * blockIdx.x / gridDim.x);
+  it.u1 = static_cast<int>(U * (blockIdx.x + 1) / gridDim.x);
   it.done = it.u >= it.u1;
   if (!it.done) unit_begin(a, it);
 }
@@ -219,11 +240,11 @@ struct __align__(16) Meta {
 
 template <typename T, int D, int G>
 struct FusedSmem {
-  using C = DecodeTile<T, D, kCW>;
+  using C = DecodeTile<T, D, Groups<G>::RW>;
   static constexpr int STAGE = C::STAGE;
   static constexpr int up16(int x) { return (x + 15) & ~15; }
   // regions after the stage ring (NS * STAGE, chosen at launch)
-  static constexpr int RED = up16(kCW * G * (D + 2) * 4);       // warp states / merge sums
+  static constexpr int RED = up16(kCW * G * (D + 2) * 4);       // warp states
   static constexpr int SEL = (kMaxK + 4) * 4 * 2;               // selected prefix + starts
   static constexpr int MISC = 1024;
   static size_t bytes(int NS) { return size_t(NS) * STAGE + RED + SEL + MISC; }
@@ -261,10 +282,10 @@ __device__ __forceinline__ void load_q_smem(const float* qs, float scale_log2,
 // Stages one item into `stg`: bulk copies that complete on `bar`, whose
 // transaction count is armed with the item's bytes.  Selected rows need the
 // selection, which the caller has waited for.
-template <typename T, int D>
+template <typename T, int D, int RW>
 __device__ void issue_item(const FusedArgs& a, const Item& item, char* stg, uint64_t* bar,
                            Meta* meta, int* sel_pref, int* sel_phys, int* sel_bh) {
-  using C = DecodeTile<T, D, kCW>;
+  using C = DecodeTile<T, D, RW>;
   const int lane = threadIdx.x & 31;
   const int* pref;
   const int* phys;
@@ -348,11 +369,11 @@ __device__ void issue_item(const FusedArgs& a, const Item& item, char* stg, uint
 }
 
 // Warp 0: stage every item of this CTA, in order, into the stage ring.
-template <typename T, int D>
+template <typename T, int D, int RW>
 __device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64_t* full,
                                         uint64_t* empty, Meta* meta, int* sel_pref,
                                         int* sel_phys, volatile int* abort_flag) {
-  using C = DecodeTile<T, D, kCW>;
+  using C = DecodeTile<T, D, RW>;
   const int NS = a.NS;
   Iter it;
   iter_begin(a, it);
@@ -369,7 +390,7 @@ __device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64
       asm volatile("griddepcontrol.wait;" ::: "memory");
       selection_visible = true;
     }
-    issue_item<T, D>(a, item, stages + size_t(s) * C::STAGE, &full[s], &meta[s], sel_pref,
+    issue_item<T, D, RW>(a, item, stages + size_t(s) * C::STAGE, &full[s], &meta[s], sel_pref,
                      sel_phys, &sel_bh);
     ++j;
     if (++s == NS) {
@@ -388,7 +409,10 @@ __device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
-  using C = DecodeTile<T, D, kCW>;
+  constexpr int HS = Groups<G>::HS, RW = Groups<G>::RW;
+  constexpr int kSlotFloats = slot_floats(G, D);
+  static_assert((kSlotFloats * 4) % 16 == 0, "bulk copies move 16-byte multiples");
+  using C = DecodeTile<T, D, RW>;
   using S = FusedSmem<T, D, G>;
   extern __shared__ __align__(128) char smem[];
   const int NS = a.NS;
@@ -402,7 +426,8 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   Meta* meta = reinterpret_cast<Meta*>(empty + kMaxStages);         // [kMaxStages]
   int* s_misc = reinterpret_cast<int*>(meta + kMaxStages);          // [16]
   volatile int* abort_flag = s_misc + 16;                           // [4]
-  float* s_f = reinterpret_cast<float*>(s_misc + 20);               // [32]
+  uint64_t* merge_bar = reinterpret_cast<uint64_t*>(s_misc + 84);   // [1] (s_f is [64] at +20)
+  float* s_f = reinterpret_cast<float*>(s_misc + 20);               // [64]
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
@@ -410,17 +435,20 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCW);
     }
+    mbar_init(merge_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   __syncthreads();
   if (warp == 0) {
-    produce<T, D>(a, stages, full, empty, meta, sel_pref, sel_phys, abort_flag);
+    produce<T, D, RW>(a, stages, full, empty, meta, sel_pref, sel_phys, abort_flag);
     return;
   }
   // ---- compute warps from here on (named barrier 1; no __syncthreads)
   const int cw = warp - 1, tid = ctid();
+  const int grp = cw / RW, rw = cw % RW;  // head group, warp within the group
+  const int g0 = grp * HS;                // first q head of this warp
 
   // item i of this CTA sits in stage s with parity ph
   int s = 0;
@@ -453,21 +481,51 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   bool have = next_item<C::TT>(a, it, item);
 
   // ---- attention over this CTA's rows, head by head
-  LaneState<T, D, G> st;
+  LaneState<T, D, HS> st;
   int cur_bh = -1;
   int ord = 0;  // part index of head cur_bh held by this CTA (its slot)
+  uint32_t merge_ph = 0;  // phase parity of merge_bar
+  float* fac = s_f;         // [G][nw] factors exp2(m_w - M) of the nw warp states
+  float* gmax = s_f + 60;   // [G] the max M
+  // fac / gmax from nw per-warp states red[w][g][m, l, o[D]]
+  auto combine = [&](int nw) {
+    if (tid < G * nw) {
+      const int gg = tid / nw, w = tid % nw;
+      float M = -INFINITY;
+      for (int v = 0; v < nw; ++v) M = fmaxf(M, red[(v * G + gg) * (D + 2)]);
+      const float mw = red[(w * G + gg) * (D + 2)];
+      fac[tid] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+      if (w == 0) gmax[gg] = M;
+    }
+  };
+  // output (and lse) of head cur_bh from nw warp states combined by fac
+  auto write_out = [&](int nw) {
+    const int b = cur_bh / a.at.Hkv, h = cur_bh % a.at.Hkv;
+    for (int x = tid; x < G * D; x += kCT) {
+      const int gg = x / D, d = x % D;
+      float num = 0.f, den = 0.f;
+      for (int w = 0; w < nw; ++w) {
+        const float f = fac[gg * nw + w];
+        num += red[(w * G + gg) * (D + 2) + 2 + d] * f;
+        den += red[(w * G + gg) * (D + 2) + 1] * f;
+      }
+      a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = den > 0.f ? num / den : 0.f;
+      if (d == 0 && a.at.lse != nullptr)
+        a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
+            den > 0.f ? (gmax[gg] + log2f(den)) * 0.6931471805599453f : -INFINITY;
+    }
+  };
   while (true) {
     const bool more = have;
     if (cur_bh >= 0 && (!more || item.bh != cur_bh)) {
-      // ---- this CTA's state of head cur_bh -> its slot; the last
-      // contributor of the head merges all of its slots
-      merge_slots<T, D, G>(st);
+      // ---- this CTA's state of head cur_bh: warp states -> red[rw][g]
+      merge_slots<T, D, HS>(st);
       const int slot_lane = lane / C::LPR, part = lane % C::LPR;
       const int rot = lane_rot<T, D>(part);
       if (slot_lane == 0) {
 #pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-          float* r = red + (cw * G + gg) * (D + 2);
+        for (int gg = 0; gg < HS; ++gg) {
+          float* r = red + (rw * G + g0 + gg) * (D + 2);
           if (part == 0) {
             r[0] = st.m[gg];
             r[1] = st.l[gg];
@@ -485,46 +543,17 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
         }
       }
       compute_sync();
-      // per q head: the CTA's max over warps and each warp's factor exp2(m_w - M)
-      float* fac = s_f;         // [G][kCW]
-      float* gmax = s_f + 28;   // [G]
-      if (tid < G * kCW) {
-        const int gg = tid / kCW, w = tid % kCW;
-        float M = -INFINITY;
-#pragma unroll
-        for (int v = 0; v < kCW; ++v) M = fmaxf(M, red[(v * G + gg) * (D + 2)]);
-        const float mw = red[(w * G + gg) * (D + 2)];
-        fac[tid] = mw == -INFINITY ? 0.f : exp2f(mw - M);
-        if (w == 0) gmax[gg] = M;
-      }
+      combine(RW);
       compute_sync();
-      // output of head cur_bh from the warp states in red, combined with fac
-      auto write_out = [&]() {
-        const int b = cur_bh / a.at.Hkv, h = cur_bh % a.at.Hkv;
-        for (int x = tid; x < G * D; x += kCT) {
-          const int gg = x / D, d = x % D;
-          float num = 0.f, den = 0.f;
-#pragma unroll
-          for (int w = 0; w < kCW; ++w) {
-            const float f = fac[gg * kCW + w];
-            num += red[(w * G + gg) * (D + 2) + 2 + d] * f;
-            den += red[(w * G + gg) * (D + 2) + 1] * f;
-          }
-          a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = den > 0.f ? num / den : 0.f;
-          if (d == 0 && a.at.lse != nullptr)
-            a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
-                den > 0.f ? (gmax[gg] + log2f(den)) * 0.6931471805599453f : -INFINITY;
-        }
-      };
       if (a.m == 1) {
-        write_out();  // this CTA holds the whole head
+        write_out(RW);  // this CTA holds the whole head
       } else {
         // this CTA's state -> slot `ord` of the head; the last of the head's
         // m parts to finish merges all m slots
         const bool slot_ok = ord >= 0 && ord < a.m;
         if (!slot_ok && tid == 0) report(a.at.status, RBA_ERR_BOUNDS, kWhereFused, 4);
-        float* base = a.slots + int64_t(cur_bh) * a.m * G * (D + 2);
-        float* slot = base + int64_t(slot_ok ? ord : 0) * G * (D + 2);
+        float* base = a.slots + int64_t(cur_bh) * a.m * kSlotFloats;
+        float* slot = base + int64_t(slot_ok ? ord : 0) * kSlotFloats;
 #pragma unroll 1
         for (int x = tid; x < G * (D + 2) && slot_ok; x += kCT) {
           const int gg = x / (D + 2), c = x % (D + 2);
@@ -533,8 +562,8 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
             acc = gmax[gg];
           } else {
 #pragma unroll
-            for (int w = 0; w < kCW; ++w)
-              acc += red[(w * G + gg) * (D + 2) + c] * fac[gg * kCW + w];
+            for (int w = 0; w < RW; ++w)
+              acc += red[(w * G + gg) * (D + 2) + c] * fac[gg * RW + w];
           }
           slot[x] = acc;
         }
@@ -545,81 +574,64 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
         }
         compute_sync();
         if (s_misc[9]) {
-          // each warp folds whole slots j = cw, cw + kCW, ... into a running
-          // (max, sum, output) per q head, three slots' loads in flight at
-          // once; then the warps' states are combined through red
+          // the last part of the head merges the m slots.  The slots go to
+          // shared memory by bulk copies into the stage ring (idle: with
+          // m > 1 a CTA holds one part of one head, all of it consumed), a
+          // chunk at a time; each thread then folds every slot's (m, l, o[d])
+          // of its output elements (g, d) into a running (max, sum, output).
+          constexpr int SLOT = kSlotFloats * 4;  // a multiple of 16 bytes
           const int nl = a.m;
-          constexpr int PER = (G * D + 31) / 32;  // output elements (g, d) per lane
-          constexpr int UN = 2;
-          float O[PER], M[G], L[G];
+          const int chunk = (NS * C::STAGE) / SLOT;
+          const int b = cur_bh / a.at.Hkv, h = cur_bh % a.at.Hkv;
+          float M[2], L[2], O[2];  // elements x = tid and tid + kCT
 #pragma unroll
-          for (int e = 0; e < PER; ++e) O[e] = 0.f;
-#pragma unroll
-          for (int gg = 0; gg < G; ++gg) {
-            M[gg] = -INFINITY;
-            L[gg] = 0.f;
+          for (int r = 0; r < 2; ++r) {
+            M[r] = -INFINITY;
+            L[r] = 0.f;
+            O[r] = 0.f;
           }
-#pragma unroll 1
-          for (int j0 = cw; j0 < nl; j0 += UN * kCW) {
-            float v[UN][PER], mj[UN][G], lj[UN][G];
+          for (int j0 = 0; j0 < nl; j0 += chunk) {
+            const int n = min(chunk, nl - j0);
+            if (tid == 0) {
+              // (the compute warps' reads of the ring are ordered before the copies)
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              mbar_arrive_tx(merge_bar, uint32_t(n) * SLOT);
+              for (int j = 0; j < n; ++j)
+                bulk_g2s(stages + size_t(j) * SLOT, base + int64_t(j0 + j) * kSlotFloats, SLOT,
+                         merge_bar);
+            }
+            const bool ok = mbar_wait(merge_bar, merge_ph, abort_flag, a.at.status, 6);
+            if (!ok && tid == 0) mbar_drain(merge_bar, merge_ph);  // no copy outlives the CTA
+            merge_ph ^= 1u;
+            const float* sm = reinterpret_cast<const float*>(stages);
 #pragma unroll
-            for (int u = 0; u < UN; ++u) {
-              const int j = j0 + u * kCW;
-              const float* sp = base + int64_t(j < nl ? j : 0) * G * (D + 2);
-#pragma unroll
-              for (int gg = 0; gg < G; ++gg) {
-                mj[u][gg] = j < nl ? __ldcg(sp + gg * (D + 2)) : -INFINITY;
-                lj[u][gg] = j < nl ? __ldcg(sp + gg * (D + 2) + 1) : 0.f;
-              }
-#pragma unroll
-              for (int e = 0; e < PER; ++e) {
-                const int x = lane + 32 * e;
-                v[u][e] = j < nl && x < G * D ? __ldcg(sp + (x / D) * (D + 2) + 2 + (x % D))
-                                              : 0.f;
+            for (int r = 0; r < 2; ++r) {
+              const int x = tid + r * kCT;
+              if (!ok || x >= G * D) continue;
+              const int gg = x / D, d = x % D;
+              for (int j = 0; j < n; ++j) {
+                const float* q = sm + j * kSlotFloats + gg * (D + 2);
+                const float mj = q[0], lj = q[1], oj = q[2 + d];
+                const float mn = fmaxf(M[r], mj);
+                const float sa = M[r] == -INFINITY ? 0.f : exp2f(M[r] - mn);
+                const float sb = mj == -INFINITY ? 0.f : exp2f(mj - mn);
+                L[r] = L[r] * sa + lj * sb;
+                O[r] = O[r] * sa + oj * sb;
+                M[r] = mn;
               }
             }
-#pragma unroll
-            for (int u = 0; u < UN; ++u) {
-              float sa[G], sb[G];
-#pragma unroll
-              for (int gg = 0; gg < G; ++gg) {
-                const float mn = fmaxf(M[gg], mj[u][gg]);
-                sa[gg] = M[gg] == -INFINITY ? 0.f : exp2f(M[gg] - mn);
-                sb[gg] = mj[u][gg] == -INFINITY ? 0.f : exp2f(mj[u][gg] - mn);
-                L[gg] = L[gg] * sa[gg] + lj[u][gg] * sb[gg];
-                M[gg] = mn;
-              }
-#pragma unroll
-              for (int e = 0; e < PER; ++e) {
-                const int gg = (lane + 32 * e) / D;
-                if (gg < G) O[e] = O[e] * sa[gg] + v[u][e] * sb[gg];
-              }
-            }
+            compute_sync();  // the chunk buffer is read before the next copy
           }
 #pragma unroll
-          for (int e = 0; e < PER; ++e) {
-            const int x = lane + 32 * e;
-            if (x < G * D) red[(cw * G + x / D) * (D + 2) + 2 + x % D] = O[e];
+          for (int r = 0; r < 2; ++r) {
+            const int x = tid + r * kCT;
+            if (x >= G * D) continue;
+            const int gg = x / D, d = x % D;
+            a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = L[r] > 0.f ? O[r] / L[r] : 0.f;
+            if (d == 0 && a.at.lse != nullptr)
+              a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
+                  L[r] > 0.f ? (M[r] + log2f(L[r])) * 0.6931471805599453f : -INFINITY;
           }
-          if (lane == 0) {
-#pragma unroll
-            for (int gg = 0; gg < G; ++gg) {
-              red[(cw * G + gg) * (D + 2)] = M[gg];
-              red[(cw * G + gg) * (D + 2) + 1] = L[gg];
-            }
-          }
-          compute_sync();
-          if (tid < G * kCW) {
-            const int gg = tid / kCW, w = tid % kCW;
-            float Mx = -INFINITY;
-#pragma unroll
-            for (int q = 0; q < kCW; ++q) Mx = fmaxf(Mx, red[(q * G + gg) * (D + 2)]);
-            const float mw = red[(w * G + gg) * (D + 2)];
-            fac[tid] = mw == -INFINITY ? 0.f : exp2f(mw - Mx);
-            if (w == 0) gmax[gg] = Mx;
-          }
-          compute_sync();
-          write_out();
           if (tid == 0) a.tickets[cur_bh] = 0;  // zero again for the next call
         }
       }
@@ -630,13 +642,13 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
     if (item.bh != cur_bh) {
       cur_bh = item.bh;
       if (cur_bh == bh_att0)
-        load_q_smem<T, D, G>(q_first, a.at.scale_log2, st);
+        load_q_smem<T, D, HS>(q_first + g0 * D, a.at.scale_log2, st);
       else
-        load_q<T, D, G>(a.at, cur_bh, st);
+        load_q<T, D, HS>(a.at, cur_bh, st, g0);
       ord = it.part;
     }
     if (wait_full()) {
-      consume_tile<T, D, G, kCW>(stages + size_t(s) * C::STAGE, meta[s].nrows, st, cw);
+      consume_tile<T, D, HS, RW>(stages + size_t(s) * C::STAGE, meta[s].nrows, st, rw);
       release();
     }
     advance();
@@ -644,11 +656,13 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   }
 }
 
+constexpr size_t kMaxSmem = 227 * 1024;  // dynamic shared memory of one CTA
+
 template <typename T, int D, int G>
 int fused_stages() {
   using S = FusedSmem<T, D, G>;
   int NS = kMaxStages;
-  while (NS > 2 && S::bytes(NS) > 227 * 1024) --NS;
+  while (NS > 2 && S::bytes(NS) > kMaxSmem) --NS;
   return NS;
 }
 
@@ -657,6 +671,7 @@ template <typename T, int D, int G>
 int fused_occupancy_t() {
   using S = FusedSmem<T, D, G>;
   const size_t smem = S::bytes(fused_stages<T, D, G>());
+  if (smem > kMaxSmem) return 0;  // (large fp32 tiles) the split-K kernel runs instead
   auto kfn = decode_fused_kernel<T, D, G>;
   if (ensure_smem(reinterpret_cast<const void*>(kfn), smem) != cudaSuccess) return -1;
   int occ = 0;
@@ -749,7 +764,7 @@ size_t fused_slot_bytes(const rba_store* st, const Geometry& g, int k, int* ms) 
   int m, P;
   partition(st, g, k, &m, &P);
   if (ms) *ms = m;
-  return m > 1 ? align_up(size_t(BH) * m * G * (d.head_dim + 2) * 4, 256) : 0;
+  return m > 1 ? align_up(size_t(BH) * m * slot_floats(G, d.head_dim) * 4, 256) : 0;
 }
 
 size_t fused_sync_bytes(const rba_store* st) {
@@ -765,6 +780,9 @@ bool fused_eligible(const rba_store* st, const Geometry& g, int k) {
   if (G != 1 && G != 2 && G != 4) return false;
   if (k > kMaxK) return false;
   if (attention_rows(st, g, k) == 0) return false;
+  const int64_t BH = int64_t(d.batch) * d.n_kv_heads;
+  if (BH >= (int64_t(1) << 24)) return false;
+  if (attention_rows(st, g, k) / BH >= (int64_t(1) << 31)) return false;
   int ms = 0;
   fused_slot_bytes(st, g, k, &ms);
   return ms <= kMaxGrid;
@@ -824,6 +842,13 @@ rba_status launch_fused(const rba_store* st, const void* q, int k, const Geometr
   a.L_st = static_cast<int>(g.sink_end + (g.T - g.w0));
   a.U_sel = k > 0 ? k * d.block_size : 0;
   fused_slot_bytes(st, g, k, &a.m);
+  // part boundaries (host side: no 64-bit divisions on the device)
+  const int64_t Lh = int64_t(a.L_st) + a.U_sel;
+  for (int c = 0; c <= a.m; ++c) {
+    const int64_t x = Lh * c / a.m;
+    a.px[c] = static_cast<int>(x);
+    a.ps[c] = static_cast<int>(x * a.L_st / Lh);
+  }
   const int G = d.n_q_heads / d.n_kv_heads;
 #define RBA_FUSED(T_, D_)                                               \
   switch (G) {                                                          \

@@ -41,7 +41,10 @@ def test_fused_step_equals_three_launches(rba, name):
     idx3 = rba.topk(scores.reshape(-1, nc), w.top_k, index_base=first).reshape(
         w.batch, w.n_kv_heads, w.top_k)
     out3, lse3 = st.attend(q, idx3, w.context, w.sink, w.window)
-    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 1
+    plan = st.decode_plan(w.top_k, w.context, w.sink, w.window)
+    # bf16 always takes the persistent kernel; fp32 with one q head per kv head
+    # has tiles too large for shared memory and runs split-K (plan -2)
+    assert plan == 1 if w.dtype == "bf16" else plan in (1, -2), plan
     ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)
     vmax = float(st.v.float().abs().max())
     for rep in range(3):
