@@ -70,6 +70,8 @@ def parse(argv=None):
     ap.add_argument("--config-seconds", type=float, default=0.5,
                     help="timed GPU seconds per extra config")
     ap.add_argument("--workload", default=WORKLOAD, help=argparse.SUPPRESS)
+    # measure one entry of the configs block only (for profiling runs)
+    ap.add_argument("--only-config", default=None, help=argparse.SUPPRESS)
     ap.add_argument("--replicas", type=int, default=0, help=argparse.SUPPRESS)
     return ap.parse_args(argv)
 
@@ -822,6 +824,17 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse(argv)
+    if args.only_config:
+        import torch
+        torch.cuda.set_device(0)
+        dev = torch.device("cuda", 0)
+        from retrieval_block_sparse_b200 import synth
+        w = synth.WORKLOADS[args.only_config]
+        fn = measure_decode_config if isinstance(w, synth.DecodeWorkload) else \
+            measure_prefill_config
+        print(json.dumps({"config": fn(args.only_config, dev, args.config_seconds, peaks())}),
+              flush=True)
+        return
     line = run_reference(args) if args.impl == "reference" else run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
