@@ -5,17 +5,22 @@
 // window of the memory) and causally to its own chunk, in one softmax;
 // 2.3.4: the retrieved window is k * block size.
 //
-// One CTA = one (chunk, q head, 128 query rows):
-//   warp 4      TMA producer: the Q tile once, then K/V tiles of 128 keys
+// One CTA = one (chunk, q head, 256 query rows) = two 128-row query tiles A
+// and B that share every K/V tile (half the K/V traffic per FLOP):
+//   warp 8      TMA producer: both Q tiles once, then K/V tiles of 128 keys
 //               (128B-swizzled) into a two-stage ring;
-//   warp 5      MMA issuer (one lane): S = Q K^T into one of two TMEM S
-//               buffers, then O += P V into the TMEM O accumulator
-//               (tcgen05.mma kind::f16, bf16 in, fp32 accumulate);
-//   warps 0-3   softmax: thread t owns query row t; reads its S row from
-//               TMEM, keeps the running max / sum, writes P (bf16) to shared
-//               memory in the operand layout, rescales its O row in TMEM
-//               when the max grows by more than 2^8, and at the end
-//               normalises O into the output.
+//   warp 9      MMA issuer (one lane): S_X = Q_X K^T into TMEM, then
+//               O_X += P_X V with P_X read from TMEM (tcgen05.mma kind::f16,
+//               bf16 in, fp32 accumulate), alternating between the tiles so
+//               the tensor core works on one tile while the other's softmax
+//               runs;
+//   warps 0-3 / 4-7   softmax of tile A / B: thread t owns query row t; two
+//               passes over its S row in 32-column chunks (max, then
+//               exp2(scale s - m) packed to bf16 and stored back over the S
+//               columns as P); O rows are rescaled in TMEM when the max grows
+//               by more than 2^8; at the end O is normalised into the output.
+// TMEM: S_A / P_A columns [0,128), S_B / P_B [128,256), O_A [256,384),
+// O_B [384,512).
 // Past blocks shorter than a tile (token-level retrieval) are first gathered
 // into a contiguous staging buffer so that every tile is one TMA box.
 // All waits on mbarriers are bounded; on expiry the kernel records
@@ -29,11 +34,11 @@
 namespace rba {
 namespace {
 
-constexpr int kBM = 128;   // query rows per CTA
+constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;   // keys per tile
 constexpr int kHD = 128;   // head dim (bf16)
 constexpr int kMaxTiles = 320;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // 8 softmax warps, TMA warp, MMA warp
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 enum MapId { kPool = 0, kStage = 1, kChunk = 2 };
@@ -52,11 +57,10 @@ struct PrefillArgs {
 };
 
 // shared memory map (bytes, from a 1024-aligned base)
-constexpr int kQOff = 0;                       // Q  [2][128][128B]
-constexpr int kKVOff = 32768;                  // 2 stages x (K [2][128][128B], V same)
+constexpr int kQOff = 0;                       // Q_A, Q_B  [2][2][128][128B]
+constexpr int kKVOff = 65536;                  // 2 stages x (K [2][128][128B], V same)
 constexpr int kStageBytes = 65536;
-constexpr int kPOff = kKVOff + 2 * kStageBytes;  // P  [2][128][128B]
-constexpr int kTileOff = kPOff + 32768;          // tile list int4[kMaxTiles]
+constexpr int kTileOff = kKVOff + 2 * kStageBytes;  // tile list int4[kMaxTiles]
 constexpr int kBarOff = kTileOff + kMaxTiles * 16;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers, + alignment slack
 
@@ -64,10 +68,9 @@ struct Bars {
   uint64_t q_full;
   uint64_t kv_full[2];
   uint64_t kv_empty[2];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t p_full;
-  uint64_t pv_done;
+  uint64_t s_full[2];   // per query tile: S = Q K^T landed in TMEM
+  uint64_t p_full[2];   // per query tile: P written to TMEM (128 arrivals)
+  uint64_t o_done[2];   // per query tile: P V accumulated into O
   uint32_t tmem_base;
   int n_tiles;
   int abort;
@@ -158,6 +161,16 @@ __device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, 
       "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(0u)
       : "memory");
 }
+// D (TMEM) += A (TMEM: M rows in lanes, K elements packed two per column) x B (smem)
+__device__ __forceinline__ void umma_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(
+          tmem_d),
+      "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -195,6 +208,21 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+// 2^x by the MUFU unit (PTX ex2.approx.ftz)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -271,15 +299,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   char* sQ = smem + kQOff;
-  char* sP = smem + kPOff;
   int4* tiles = reinterpret_cast<int4*>(smem + kTileOff);
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, hq = blockIdx.y, c = blockIdx.z;
+  const int pt = blockIdx.x, hq = blockIdx.y, c = blockIdx.z;
   const int h = hq / a.G;
+  // query tiles of this CTA: X = 0 (A) rows [256 pt, +128), X = 1 (B) the next 128
+  const int qt0 = 2 * pt;
+  const bool has_b = (qt0 + 1) * kBM < a.Nq;
+  const int qt_last = has_b ? qt0 + 1 : qt0;
+  // key tile j is active for query tile X unless it is an own-chunk tile past X's diagonal
+  auto active = [&](const int4& t, int X) { return t.w < 0 || t.w <= qt0 + X; };
 
-  if (warp == 4) {
-    const int n = build_tiles(a, c, h, qt, tiles);
+  if (warp == 8) {
+    const int n = build_tiles(a, c, h, qt_last, tiles);
     if (lane == 0) {
       bars->n_tiles = n;
       bars->abort = 0;
@@ -288,15 +321,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars->kv_full[s], 1);
         mbar_init(&bars->kv_empty[s], 1);
         mbar_init(&bars->s_full[s], 1);
-        mbar_init(&bars->s_free[s], 128);
+        mbar_init(&bars->p_full[s], 128);
+        mbar_init(&bars->o_done[s], 1);
       }
-      mbar_init(&bars->p_full, 128);
-      mbar_init(&bars->pv_done, 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
   }
-  if (warp == 5) {  // TMEM: S buffers at columns [0,128) and [128,256), O at [256,384)
+  if (warp == 9) {  // TMEM: S/P of A [0,128), of B [128,256); O_A [256,384), O_B [384,512)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&bars->tmem_base)),
                  "r"(512u)
@@ -309,13 +341,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   const int n = bars->n_tiles;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      mbar_arrive_tx(&bars->q_full, 32768);
-      const int qrow = (c * a.Hq + hq) * a.Nq + qt * kBM;
+      mbar_arrive_tx(&bars->q_full, has_b ? 65536 : 32768);
+      const int qrow = (c * a.Hq + hq) * a.Nq + qt0 * kBM;
       tma_load_2d(sQ, &map_q, 0, qrow, &bars->q_full);
       tma_load_2d(sQ + 16384, &map_q, 64, qrow, &bars->q_full);
+      if (has_b) {
+        tma_load_2d(sQ + 32768, &map_q, 0, qrow + kBM, &bars->q_full);
+        tma_load_2d(sQ + 49152, &map_q, 64, qrow + kBM, &bars->q_full);
+      }
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j & 1;
@@ -339,146 +375,176 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16(0), id_pv = idesc_bf16(1);
       bool ok = mbar_wait(&bars->q_full, 0, bars, a.status, 2);
-      const uint32_t q_base = smem_u32(sQ), p_base = smem_u32(sP);
-      int n_qk = 0, n_pv = 0;  // MMAs committed (for the drain at exit)
-      auto issue_pv = [&](int jj) {
-        const int st = jj & 1;
-        const uint32_t v_base = smem_u32(smem + kKVOff + st * kStageBytes + 32768);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // A = P (K-major, keys contiguous); B = V (MN-major: head dim contiguous)
-          const uint64_t da = sdesc(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 1, 64);
-          const uint64_t db = sdesc(v_base + kk * 2048, 1024, 64);
-          umma(tmem + 256, da, db, id_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars->pv_done);
-        umma_commit(&bars->kv_empty[st]);
-        ++n_pv;
+      const int nx = has_b ? 2 : 1;
+      int n_pv[2] = {0, 0};     // P V issued per query tile (o_done phases)
+      int n_qk[2] = {0, 0};     // Q K^T issued per query tile (s_full phases)
+      int n_commit = 0;         // commits of kv_empty
+      int kv_seen = -1;         // last key tile whose K/V was waited for
+      auto wait_kv = [&](int j) -> bool {
+        if (j <= kv_seen) return true;
+        kv_seen = j;
+        return mbar_wait(&bars->kv_full[j & 1], (j >> 1) & 1, bars, a.status, 3);
       };
-      for (int j = 0; j < n && ok; ++j) {
-        const int st = j & 1, sb = j & 1;
-        if (!mbar_wait(&bars->kv_full[st], (j >> 1) & 1, bars, a.status, 3)) break;
-        if (j >= 2 && !mbar_wait(&bars->s_free[sb], ((j >> 1) - 1) & 1, bars, a.status, 4)) break;
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(smem + kKVOff + st * kStageBytes);
+      auto issue_qk = [&](int j, int X) {
+        const uint32_t q_base = smem_u32(sQ + X * 32768);
+        const uint32_t k_base = smem_u32(smem + kKVOff + (j & 1) * kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
           const uint64_t da = sdesc(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 1, 64);
           const uint64_t db = sdesc(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 1, 64);
-          umma(tmem + sb * 128, da, db, id_qk, kk > 0 ? 1u : 0u);
+          umma(tmem + X * 128, da, db, id_qk, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->s_full[sb]);
-        ++n_qk;
-        if (j >= 1) {
-          if (!mbar_wait(&bars->p_full, (j - 1) & 1, bars, a.status, 5)) break;
+        umma_commit(&bars->s_full[X]);
+        ++n_qk[X];
+      };
+      // first tile: S for both query tiles
+      if (ok && n > 0) ok = wait_kv(0);
+      for (int X = 0; X < nx && ok; ++X)
+        if (active(tiles[0], X)) issue_qk(0, X);
+      for (int j = 0; j < n && ok; ++j) {
+        const int4 t = tiles[j];
+        const uint32_t v_base = smem_u32(smem + kKVOff + (j & 1) * kStageBytes + 32768);
+        int last_x = -1;
+        for (int X = 0; X < nx; ++X)
+          if (active(t, X)) last_x = X;
+        for (int X = 0; X < nx && ok; ++X) {
+          if (!active(t, X)) continue;
+          // O_X += P_X V once the softmax has written P_X
+          if (!mbar_wait(&bars->p_full[X], n_pv[X] & 1, bars, a.status, 5)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          issue_pv(j - 1);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // A = P (TMEM, 16 keys = 8 columns per step); B = V (MN-major)
+            const uint64_t db = sdesc(v_base + kk * 2048, 1024, 64);
+            umma_ta(tmem + 256 + X * 128, tmem + X * 128 + kk * 8, db, id_pv,
+                    (n_pv[X] > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->o_done[X]);
+          ++n_pv[X];
+          if (X == last_x) {
+            umma_commit(&bars->kv_empty[j & 1]);
+            ++n_commit;
+          }
+          // next S_X overwrites P_X: after this P V has completed
+          if (j + 1 < n && active(tiles[j + 1], X)) {
+            if (!wait_kv(j + 1) ||
+                !mbar_wait(&bars->o_done[X], (n_pv[X] - 1) & 1, bars, a.status, 4)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_qk(j + 1, X);
+          }
         }
-      }
-      if (n > 0 && !bars->abort && mbar_wait(&bars->p_full, (n - 1) & 1, bars, a.status, 6)) {
-        tc_fence_after();
-        issue_pv(n - 1);
       }
       if (bars->abort) {  // no MMA may still be running when TMEM is freed
-        if (n_qk > 0) mbar_drain(&bars->s_full[(n_qk - 1) & 1], ((n_qk - 1) >> 1) & 1);
-        if (n_pv > 0) mbar_drain(&bars->pv_done, (n_pv - 1) & 1);
+        for (int X = 0; X < nx; ++X) {
+          if (n_qk[X] > 0) mbar_drain(&bars->s_full[X], (n_qk[X] - 1) & 1);
+          if (n_pv[X] > 0) mbar_drain(&bars->o_done[X], (n_pv[X] - 1) & 1);
+        }
       }
+      (void)n_commit;
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = tid;  // query row within the tile (TMEM lane)
-    const int qpos = qt * kBM + r;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    // tcgen05.ld / st are warp-collective: every decision that guards one
-    // is made uniform across the warp (__all_sync / __any_sync)
+    const int X = warp >> 2;                       // query tile of this warpgroup
+    const int r = tid & 127;                       // query row within the tile (TMEM lane)
+    const int qpos = (qt0 + X) * kBM + r;
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t s_col = X * 128, o_col = 256 + X * 128;
+    float m = -INFINITY, l = 0.f;  // running max (scaled log2 units) and sum
+    bool ok = X == 0 || has_b;
+    int n_s = 0;
     for (int j = 0; j < n && ok; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (j >> 1) & 1, bars, a.status, 7))) {
+      const int4 t = tiles[j];
+      if (!active(t, X)) continue;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[X], n_s & 1, bars, a.status, 7))) {
         ok = false;
         break;
       }
+      ++n_s;
       tc_fence_after();
-      float s[kBN];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tmem + lane_off + sb * 128 + q4 * 32, s + q4 * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->s_free[sb]);
-      const int4 t = tiles[j];
       const int valid = t.z;
       const int lim = t.w >= 0 ? min(valid, qpos - t.w * kBN + 1) : valid;  // keys [0, lim) visible
+      // pass 1: the row's max over its visible keys
       float mt = -INFINITY;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float v[32];
+        tmem_ld32(tmem + lane_off + s_col + q4 * 32, v);
+        tmem_wait_ld();
+        if (lim >= (q4 + 1) * 32) {
 #pragma unroll
-      for (int x = 0; x < kBN; ++x) {
-        s[x] = x < lim ? s[x] * a.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[x]);
+          for (int x = 0; x < 32; ++x) mt = fmaxf(mt, v[x]);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if (q4 * 32 + x < lim) mt = fmaxf(mt, v[x]);
+        }
       }
-      const float m_new = fmaxf(m, mt);
-      const bool rescale = m_new > m + 8.f;  // also when m is still -inf
+      const float m_new = fmaxf(m, mt * a.scale_log2);
+      const bool rescale = m_new > m + 8.f;  // lazy: also when m is still -inf
       const float m_use = rescale ? m_new : m;
-      float rs = 0.f;
-      uint32_t pk[kBN / 2];
-#pragma unroll
-      for (int x = 0; x < kBN; x += 2) {
-        const float p0 = m_use == -INFINITY ? 0.f : exp2f(s[x] - m_use);
-        const float p1 = m_use == -INFINITY ? 0.f : exp2f(s[x + 1] - m_use);
-        rs += p0 + p1;
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-        pk[x / 2] = *reinterpret_cast<const uint32_t*>(&b2);
-      }
       const float corr = (rescale && m != -INFINITY) ? exp2f(m - m_use) : 1.f;
-      l = l * corr + rs;
-      // P buffer and O are free once the previous P V has completed
-      if (j >= 1 &&
-          !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (j - 1) & 1, bars, a.status, 8))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // rows whose max grew rescale their O row; the warp loads and stores
-      // together (corr is 1 for the other rows)
-      if (j >= 1 && __any_sync(0xffffffffu, rescale && corr != 1.f)) {
+      // O rows whose max grew are rescaled; the warp loads and stores together
+      // (O_X is idle: the next S_X was issued only after the last P_X V)
+      if (__any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) {
           float o[32];
-          tmem_ld32(tmem + lane_off + 256 + q4 * 32, o);
+          tmem_ld32(tmem + lane_off + o_col + q4 * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[x] *= corr;
-          tmem_st32(tmem + lane_off + 256 + q4 * 32, o);
+          tmem_st32(tmem + lane_off + o_col + q4 * 32, o);
         }
-        tmem_wait_st();
       }
-      // P row r into the K-major 128B-swizzled operand layout
+      // pass 2: P = exp2(scale s - m), bf16 pairs stored over the S columns
+      const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
+      float rs = 0.f;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float v[32];
+        tmem_ld32(tmem + lane_off + s_col + q4 * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int kb = ch >> 3, cc = ch & 7;
-        char* dst = sP + kb * 16384 + r * 128 + ((cc ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) =
-            make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+        for (int x = 0; x < 32; x += 2) {
+          const bool in0 = q4 * 32 + x < lim && m_use != -INFINITY;
+          const bool in1 = q4 * 32 + x + 1 < lim && m_use != -INFINITY;
+          const float p0 = in0 ? ex2_approx(fmaf(v[x], a.scale_log2, neg_m)) : 0.f;
+          const float p1 = in1 ? ex2_approx(fmaf(v[x + 1], a.scale_log2, neg_m)) : 0.f;
+          rs += p0 + p1;
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          pk[x / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        tmem_st16(tmem + lane_off + s_col + q4 * 16, pk);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      tmem_wait_st();
+      l = l * corr + rs;
       m = m_use;
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[X]);
     }
-    if (ok && n > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&bars->pv_done, (n - 1) & 1, bars, a.status, 9))) {
+    // final: O / l into the output once the last P V has completed
+    if (ok && n_s > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], (n_s - 1) & 1, bars, a.status, 9))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       float* orow = a.out + ((int64_t(c) * a.Hq + hq) * a.Nq + qpos) * kHD;
 #pragma unroll 1
       for (int q4 = 0; q4 < 4; ++q4) {
         float o[32];
-        tmem_ld32(tmem + lane_off + 256 + q4 * 32, o);  // whole warp, rows past Nq too
+        tmem_ld32(tmem + lane_off + o_col + q4 * 32, o);  // whole warp, rows past Nq too
         tmem_wait_ld();
         if (qpos < a.Nq) {
 #pragma unroll
@@ -487,20 +553,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_float4(o[x] * inv, o[x + 1] * inv, o[x + 2] * inv, o[x + 3] * inv);
         }
       }
-      if (qpos < a.Nq) {
-        if (a.lse != nullptr)
-          a.lse[(int64_t(c) * a.Hq + hq) * a.Nq + qpos] =
-              l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
-      }
-    } else if (n == 0 && qpos < a.Nq) {
-      float* orow = a.out + ((int64_t(c) * a.Hq + hq) * a.Nq + qpos) * kHD;
-      for (int x = 0; x < kHD; ++x) orow[x] = 0.f;
-      if (a.lse != nullptr) a.lse[(int64_t(c) * a.Hq + hq) * a.Nq + qpos] = -INFINITY;
+      if (qpos < a.Nq && a.lse != nullptr)
+        a.lse[(int64_t(c) * a.Hq + hq) * a.Nq + qpos] =
+            l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u)
                  : "memory");
@@ -708,7 +768,7 @@ rba_status rba_attend_prefill(const rba_store* st, const void* q, int32_t n_chun
     msv = mpv;
   }
   RBA_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(prefill_kernel), kSmemBytes));
-  const dim3 grid(static_cast<unsigned>((chunk_len + kBM - 1) / kBM),
+  const dim3 grid(static_cast<unsigned>((chunk_len + 2 * kBM - 1) / (2 * kBM)),
                   static_cast<unsigned>(d.n_q_heads), static_cast<unsigned>(n_chunks));
   prefill_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a, mq, mpk, mpv, msk, msv, mck, mcv);
   RBA_LAUNCH_CHECK();
