@@ -483,8 +483,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_off + s_col + q4 * 32, v);
         tmem_wait_ld();
         if (lim >= (q4 + 1) * 32) {
+          float m2 = mt;
 #pragma unroll
-          for (int x = 0; x < 32; ++x) mt = fmaxf(mt, v[x]);
+          for (int x = 0; x < 32; x += 2) {  // two chains
+            mt = fmaxf(mt, v[x]);
+            m2 = fmaxf(m2, v[x + 1]);
+          }
+          mt = fmaxf(mt, m2);
         } else {
 #pragma unroll
           for (int x = 0; x < 32; ++x)
@@ -509,27 +514,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // pass 2: P = exp2(scale s - m), bf16 pairs stored over the S columns
+      // (pairs through f32x2 FMA / add; masks only where keys are cut off)
       const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
-      float rs = 0.f;
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      const bool whole = lim >= kBN && m_use != -INFINITY;  // no key of this tile is masked
+      float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll 1
       for (int q4 = 0; q4 < 4; ++q4) {
         float v[32];
         tmem_ld32(tmem + lane_off + s_col + q4 * 32, v);
         tmem_wait_ld();
         uint32_t pk[16];
+        if (whole) {
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const bool in0 = q4 * 32 + x < lim && m_use != -INFINITY;
-          const bool in1 = q4 * 32 + x + 1 < lim && m_use != -INFINITY;
-          const float p0 = in0 ? ex2_approx(fmaf(v[x], a.scale_log2, neg_m)) : 0.f;
-          const float p1 = in1 ? ex2_approx(fmaf(v[x + 1], a.scale_log2, neg_m)) : 0.f;
-          rs += p0 + p1;
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          pk[x / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+          for (int x = 0; x < 32; x += 2) {
+            const float2 e = __ffma2_rn(make_float2(v[x], v[x + 1]), sc2, nm2);
+            const float2 pp = make_float2(ex2_approx(e.x), ex2_approx(e.y));
+            rs2 = __fadd2_rn(rs2, pp);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(pp.x, pp.y);
+            pk[x / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            const bool in0 = q4 * 32 + x < lim && m_use != -INFINITY;
+            const bool in1 = q4 * 32 + x + 1 < lim && m_use != -INFINITY;
+            const float2 e = __ffma2_rn(make_float2(v[x], v[x + 1]), sc2, nm2);
+            const float2 pp = make_float2(in0 ? ex2_approx(e.x) : 0.f, in1 ? ex2_approx(e.y) : 0.f);
+            rs2 = __fadd2_rn(rs2, pp);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(pp.x, pp.y);
+            pk[x / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
         }
         tmem_st16(tmem + lane_off + s_col + q4 * 16, pk);
       }
       tmem_wait_st();
+      const float rs = rs2.x + rs2.y;
       l = l * corr + rs;
       m = m_use;
       tc_fence_before();
