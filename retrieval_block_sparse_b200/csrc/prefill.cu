@@ -224,6 +224,19 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// The registers of an in-flight tcgen05.ld pass through this empty asm after
+// tcgen05.wait::ld, so the compiler cannot move their uses above the wait.
+__device__ __forceinline__ void tmem_regs_ready(float* v) {
+  asm volatile(""
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                 "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]),
+                 "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]),
+                 "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]),
+                 "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]),
+                 "+f"(v[30]), "+f"(v[31])
+               :
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -475,25 +488,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int valid = t.z;
       const int lim = t.w >= 0 ? min(valid, qpos - t.w * kBN + 1) : valid;  // keys [0, lim) visible
-      // pass 1: the row's max over its visible keys
+      // pass 1: the row's max over its visible keys (two chunks in flight per wait)
       float mt = -INFINITY;
 #pragma unroll 1
-      for (int q4 = 0; q4 < 4; ++q4) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + s_col + q4 * 32, v);
+      for (int q8 = 0; q8 < 4; q8 += 2) {
+        float va[32], vb[32];
+        tmem_ld32(tmem + lane_off + s_col + q8 * 32, va);
+        tmem_ld32(tmem + lane_off + s_col + (q8 + 1) * 32, vb);
         tmem_wait_ld();
-        if (lim >= (q4 + 1) * 32) {
+        tmem_regs_ready(va);
+        tmem_regs_ready(vb);
+        if (lim >= (q8 + 2) * 32) {
           float m2 = mt;
 #pragma unroll
-          for (int x = 0; x < 32; x += 2) {  // two chains
-            mt = fmaxf(mt, v[x]);
-            m2 = fmaxf(m2, v[x + 1]);
+          for (int x = 0; x < 32; ++x) {  // two chains
+            mt = fmaxf(mt, va[x]);
+            m2 = fmaxf(m2, vb[x]);
           }
           mt = fmaxf(mt, m2);
         } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (q4 * 32 + x < lim) mt = fmaxf(mt, v[x]);
+          for (int x = 0; x < 32; ++x) {
+            if (q8 * 32 + x < lim) mt = fmaxf(mt, va[x]);
+            if ((q8 + 1) * 32 + x < lim) mt = fmaxf(mt, vb[x]);
+          }
         }
       }
       const float m_new = fmaxf(m, mt * a.scale_log2);
@@ -508,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float o[32];
           tmem_ld32(tmem + lane_off + o_col + q4 * 32, o);
           tmem_wait_ld();
+          tmem_regs_ready(o);
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[x] *= corr;
           tmem_st32(tmem + lane_off + o_col + q4 * 32, o);
@@ -520,11 +539,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 nm2 = make_float2(neg_m, neg_m);
       const bool whole = lim >= kBN && m_use != -INFINITY;  // no key of this tile is masked
       float2 rs2 = make_float2(0.f, 0.f);
-#pragma unroll 1
+      // chunk q4 + 1 is loaded while chunk q4 is exponentiated (P chunk q4 goes to
+      // columns [16 q4, 16 q4 + 16), below every chunk still to be read)
+      float vbuf[2][32];
+      tmem_ld32(tmem + lane_off + s_col, vbuf[0]);
+      tmem_wait_ld();
+      tmem_regs_ready(vbuf[0]);
+#pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + s_col + q4 * 32, v);
-        tmem_wait_ld();
+        const float* v = vbuf[q4 & 1];
+        if (q4 < 3) tmem_ld32(tmem + lane_off + s_col + (q4 + 1) * 32, vbuf[(q4 + 1) & 1]);
         uint32_t pk[16];
         if (whole) {
 #pragma unroll
@@ -548,6 +572,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tmem_st16(tmem + lane_off + s_col + q4 * 16, pk);
+        if (q4 < 3) {
+          tmem_wait_ld();
+          tmem_regs_ready(vbuf[(q4 + 1) & 1]);
+        }
       }
       tmem_wait_st();
       const float rs = rs2.x + rs2.y;
@@ -567,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float o[32];
         tmem_ld32(tmem + lane_off + o_col + q4 * 32, o);  // whole warp, rows past Nq too
         tmem_wait_ld();
+        tmem_regs_ready(o);
         if (qpos < a.Nq) {
 #pragma unroll
           for (int x = 0; x < 32; x += 4)
