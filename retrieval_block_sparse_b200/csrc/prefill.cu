@@ -538,7 +538,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
       const float2 nm2 = make_float2(neg_m, neg_m);
       const bool whole = lim >= kBN && m_use != -INFINITY;  // no key of this tile is masked
-      float2 rs2 = make_float2(0.f, 0.f);
+      float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};  // four independent sum chains
       // chunk q4 + 1 is loaded while chunk q4 is exponentiated (P chunk q4 goes to
       // columns [16 q4, 16 q4 + 16), below every chunk still to be read)
       float vbuf[2][32];
@@ -555,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int x = 0; x < 32; x += 2) {
             const float2 e = __ffma2_rn(make_float2(v[x], v[x + 1]), sc2, nm2);
             const float2 pp = make_float2(ex2_approx(e.x), ex2_approx(e.y));
-            rs2 = __fadd2_rn(rs2, pp);
+            rs2[(x >> 1) & 3] = __fadd2_rn(rs2[(x >> 1) & 3], pp);
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(pp.x, pp.y);
             pk[x / 2] = *reinterpret_cast<const uint32_t*>(&b2);
           }
@@ -566,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool in1 = q4 * 32 + x + 1 < lim && m_use != -INFINITY;
             const float2 e = __ffma2_rn(make_float2(v[x], v[x + 1]), sc2, nm2);
             const float2 pp = make_float2(in0 ? ex2_approx(e.x) : 0.f, in1 ? ex2_approx(e.y) : 0.f);
-            rs2 = __fadd2_rn(rs2, pp);
+            rs2[(x >> 1) & 3] = __fadd2_rn(rs2[(x >> 1) & 3], pp);
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(pp.x, pp.y);
             pk[x / 2] = *reinterpret_cast<const uint32_t*>(&b2);
           }
@@ -578,7 +579,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tmem_wait_st();
-      const float rs = rs2.x + rs2.y;
+      const float2 r01 = __fadd2_rn(rs2[0], rs2[1]), r23 = __fadd2_rn(rs2[2], rs2[3]);
+      const float2 r03 = __fadd2_rn(r01, r23);
+      const float rs = r03.x + r03.y;
       l = l * corr + rs;
       m = m_use;
       tc_fence_before();
