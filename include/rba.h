@@ -257,6 +257,28 @@ size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t
 int32_t rba_decode_step_plan(const rba_store* store, int32_t k, int64_t T, int32_t sink,
                              int32_t window);
 
+/* One step of streaming decode ([IL] overall framework: the newest tokens form
+ * the local window and the tokens before it stay in memory as units that are
+ * represented once; [ML] 2.3.2: a completed chunk is memorised).  The store
+ * holds T tokens.  The call
+ *   1. appends the new token's K and V (device dtype [B][Hkv][D]) at position T,
+ *   2. if T + 1 is a multiple of the block size, memorises block (T + 1) / bs - 1
+ *      from the pools (aux / n_aux as rba_memorize for one block: probe queries
+ *      [Hkv][n_aux][D] for RBA_REP_TOPR_ATTN, the landmark keys [B][Hkv][1][n_rep][D]
+ *      for RBA_REP_EXTERNAL, NULL for RBA_REP_MEAN and RBA_REP_IDENTITY),
+ *   3. runs rba_decode_step for q over the T + 1 tokens with k' = min(k, candidates)
+ *      blocks (written to *k_used when k_used is not NULL, host); idx is
+ *      [B][Hkv][k'], out / lse as rba_decode_step.
+ * The caller advances T by one per call.  Everything is enqueued on `stream`.
+ *   workspace >= rba_decode_step_workspace_size(store, k, T + 1, sink, window).
+ * Errors: INVALID_ARG (T + 1 above the capacity, cosine stores, invalid
+ * geometry), and those of rba_memorize and rba_decode_step. */
+rba_status rba_stream_step(rba_store* store, const void* q, const void* k_new,
+                           const void* v_new, int64_t T, int32_t k, int32_t sink, int32_t window,
+                           float scale, const void* aux, int32_t n_aux, int32_t* idx, float* out,
+                           float* lse, int32_t* k_used, void* workspace, size_t ws_bytes,
+                           cudaStream_t stream);
+
 /* rba_decode_step from and to host memory: copies q_host (host, dtype [B][Hq][D]) into
  * q_dev, runs the step, copies out/lse/idx back into the host buffers (any of lse_host,
  * idx_host may be NULL), then synchronises `stream`.  q_dev, idx_dev, out_dev, lse_dev are

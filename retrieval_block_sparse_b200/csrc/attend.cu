@@ -294,6 +294,44 @@ rba_status rba_decode_step(const rba_store* st, const void* q, int32_t k, int64_
   return attend_any(st, q, idx, k, g, scale, out, lse, w.att, fused && k > 0, stream);
 }
 
+rba_status rba_stream_step(rba_store* st, const void* q, const void* k_new, const void* v_new,
+                           int64_t T, int32_t k, int32_t sink, int32_t window, float scale,
+                           const void* aux, int32_t n_aux, int32_t* idx, float* out, float* lse,
+                           int32_t* k_used, void* workspace, size_t ws_bytes,
+                           cudaStream_t stream) {
+  using namespace rba;
+  if (st == nullptr || q == nullptr || k_new == nullptr || v_new == nullptr || T < 0 || k < 0)
+    return RBA_ERR_INVALID_ARG;
+  const rba_store_desc& d = st->d;
+  if (d.mode == RBA_REP_EMBED_COSINE) return RBA_ERR_INVALID_ARG;
+  if (T + 1 > d.capacity_tokens) return RBA_ERR_INVALID_ARG;
+  // the step's geometry first: nothing is launched if it is invalid
+  Geometry g;
+  rba_status s = geometry(st, T + 1, sink, window, &g);
+  if (s != RBA_OK) return s;
+  const int32_t ke = k < g.nc ? k : g.nc;  // early in a stream fewer blocks are candidates
+  if (k_used != nullptr) *k_used = ke;
+  // 1. the new token's K and V at position T of every (batch, kv head)
+  const size_t row = size_t(d.head_dim) * dtype_size(d.dtype);
+  const size_t rows = size_t(d.batch) * d.n_kv_heads;
+  const size_t pitch = size_t(d.capacity_tokens) * row;
+  char* kdst = static_cast<char*>(st->k) + size_t(T) * row;
+  char* vdst = static_cast<char*>(st->v) + size_t(T) * row;
+  RBA_CUDA_TRY(cudaMemcpy2DAsync(kdst, pitch, k_new, row, row, rows, cudaMemcpyDeviceToDevice,
+                                 stream));
+  RBA_CUDA_TRY(cudaMemcpy2DAsync(vdst, pitch, v_new, row, row, rows, cudaMemcpyDeviceToDevice,
+                                 stream));
+  // 2. the block this token completes becomes a memory unit: its representation
+  if ((T + 1) % d.block_size == 0 && d.mode != RBA_REP_IDENTITY) {
+    s = rba_memorize(st, nullptr, nullptr, (T + 1) / d.block_size - 1, 1, aux, n_aux, scale,
+                     stream);
+    if (s != RBA_OK) return s;
+  }
+  // 3. the decode step over the T + 1 tokens
+  return rba_decode_step(st, q, ke, T + 1, sink, window, scale, nullptr, idx, out, lse,
+                         workspace, ws_bytes, stream);
+}
+
 int32_t rba_decode_step_plan(const rba_store* st, int32_t k, int64_t T, int32_t sink,
                              int32_t window) {
   using namespace rba;

@@ -45,6 +45,8 @@ SIGNATURES = {
                                  _p, _c_size, _p]),
     "rba_decode_step_workspace_size": (_c_size, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
     "rba_decode_step_plan": (_c_i32, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
+    "rba_stream_step": (_c_i32, [_p, _p, _p, _p, _c_i64, _c_i32, _c_i32, _c_i32, _c_f32, _p,
+                                 _c_i32, _p, _p, _p, ctypes.POINTER(_c_i32), _p, _c_size, _p]),
     "rba_decode_step_host": (_c_i32, [_p, _p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32, _p, _p,
                                       _p, _p, _p, _p, _p, _c_size, _p]),
     "rba_store_check": (_c_i32, [_p, _p]),
@@ -277,6 +279,32 @@ class Store:
                                      _ptr(idx), _ptr(out), _ptr(lse), _ptr(workspace),
                                      workspace.numel(), _stream()), "rba_decode_step")
         return idx, out, lse
+
+    def stream_step(self, q, k_new, v_new, T, k, sink, window, *, aux=None, scale=None,
+                    workspace=None, out=None, lse=None, idx=None):
+        """Append one token's K/V at position T, memorise the block it completes,
+        decode q over T + 1 tokens.  Returns (idx [B][Hkv][k'], out, lse) with
+        k' = min(k, candidates at T + 1)."""
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.D)
+        dev = q.device
+        if out is None:
+            out = torch.empty((self.B, self.Hq, self.D), dtype=torch.float32, device=dev)
+        if lse is None:
+            lse = torch.empty((self.B, self.Hq), dtype=torch.float32, device=dev)
+        if idx is None:
+            idx = torch.empty((self.B, self.Hkv, max(k, 1)), dtype=torch.int32, device=dev)
+        if workspace is None:
+            workspace = self.decode_workspace(k, T + 1, sink, window)
+        n_aux = aux.shape[1] if (aux is not None and self.mode == "topr_attn") else 0
+        used = ctypes.c_int32(0)
+        _check(lib().rba_stream_step(self.handle, _ptr(q), _ptr(k_new), _ptr(v_new), T, k, sink,
+                                     window, scale, _ptr(aux), n_aux, _ptr(idx), _ptr(out),
+                                     _ptr(lse), ctypes.byref(used), _ptr(workspace),
+                                     workspace.numel(), _stream()), "rba_stream_step")
+        kk = used.value
+        sel = idx.reshape(-1)[: self.B * self.Hkv * kk].reshape(self.B, self.Hkv, kk)
+        return sel, out, lse
 
     def decode_step_host(self, q_host, k, T, sink, window, *, q_dev, idx_dev, out_dev, lse_dev,
                          out_host, lse_host=None, idx_host=None, workspace, scale=None):
