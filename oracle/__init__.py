@@ -10,4 +10,8 @@ invariants, library routines or brute force; see the docstring of each
 function for the passage of the pages it restates.
 """
 from .retrieval import *  # noqa: F401,F403
-from .retrieval import __all__  # noqa: F401
+from .retrieval import __all__ as _r_all
+from .memory import *  # noqa: F401,F403
+from .memory import __all__ as _m_all
+
+__all__ = list(_r_all) + list(_m_all)
