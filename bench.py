@@ -720,6 +720,78 @@ def measure_prefill_config(name, dev, seconds, pk):
     return res
 
 
+def measure_memory_update(name, dev, trials, pk):
+    """Dynamic memory update (MemLong section 2.3.2) of the full store of
+    workload `name`: synthetic retrieval counters, the page's 10% / 10% / 50%
+    proportions over the blocks after the sink, in-place compaction.  Each
+    trial restores the store from a copy (untimed; the copy, larger than L2,
+    also evicts it) and times one update with CUDA events on the stream.
+
+    Algorithmic bytes: every kept entry moves (the oldest entries are dropped,
+    so each kept one shifts), read + write of its K/V rows over the unit's kv
+    heads, its representation, positions and counter, plus one read of the
+    counters by the selection and the keep map written."""
+    import torch
+    import retrieval_block_sparse_b200 as rba
+    from retrieval_block_sparse_b200 import synth
+    w = synth.WORKLOADS[name]
+    cosine = getattr(w, "score_mode", "dot") == "cosine"
+    if cosine:
+        mode, r, d_ret, batch = "embed_cosine", 1, w.d_ret, 1
+    else:
+        mode, r, d_ret, batch = w.rep_mode, w.n_rep, 0, w.batch
+    st = rba.Store(batch=batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                   head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
+                   dtype=w.dtype, mode=mode, n_rep=r, d_ret=d_ret, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    for t in (st.k, st.v, st.rep):
+        if t is not None:
+            t.copy_(torch.randn(t.shape, generator=gen, device=dev, dtype=torch.float32))
+    if st.rep_pos is not None:
+        st.rep_pos.random_(0, w.block_size, generator=gen)
+    U = st.memory_units()
+    counts = synth.retrieval_counts(w.seed, U, st.cap_blocks)
+    counters = torch.from_numpy(counts.view(np.int32)).to(dev)
+    T, bs = w.context, w.block_size
+    nb = T // bs
+    pinned = -(-w.sink // bs) if w.sink else 0
+    newest, oldest, total = rba.memory_rule(nb - pinned)
+    keep_map = torch.empty((U, max(total, 1)), dtype=torch.int32, device=dev)
+    saved = [t.clone() for t in (st.k, st.v, st.rep, st.rep_pos, counters) if t is not None]
+    live = [t for t in (st.k, st.v, st.rep, st.rep_pos, counters) if t is not None]
+    stream = torch.cuda.current_stream()
+    times = []
+    for i in range(trials + 2):
+        for a, b in zip(live, saved):
+            a.copy_(b)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        t_new, _ = st.memory_update(T, counters, pinned_blocks=pinned, keep_map=keep_map)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            times.append(e0.elapsed_time(e1) * 1e3)
+    st.check()
+    es = 2 if w.dtype == "bf16" else 4
+    heads = w.n_kv_heads if cosine else 1
+    kv_b = heads * 2 * bs * w.head_dim * es
+    rep_b = 0 if st.rep is None else \
+        st.rep.numel() // (U * st.cap_blocks) * st.rep.element_size()
+    pos_b = 4 * r if st.rep_pos is not None else 0
+    moved = U * total * 2 * (kv_b + rep_b + pos_b + 4)
+    algo = moved + U * (nb - pinned - newest - oldest) * 4 + U * total * 4
+    us = float(np.median(times))
+    gbs = algo / (us * 1e-6) / 1e9
+    rounds = -(-total // max(oldest, 1))
+    return {"workload": name, "units": U, "entries": nb - pinned, "pinned_blocks": pinned,
+            "keep_newest": newest, "drop_oldest": oldest, "keep_total": total,
+            "T_new": t_new, "launches": 1 + rounds + 1, "trials": trials,
+            "update_us": round(us, 2), "algorithmic_bytes": algo,
+            "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
+            "timing": "median of trials; store restored from a copy between trials"}
+
+
 def measure_configs(dev, seconds):
     pk = peaks()
     out = {}
@@ -727,6 +799,8 @@ def measure_configs(dev, seconds):
         out[name] = measure_decode_config(name, dev, seconds, pk)
     for name in ("memlong-cosine-prefill", "token-retrieval-prefill-1m"):
         out[name] = measure_prefill_config(name, dev, seconds, pk)
+    for name in ("memlong-cosine-prefill", "infllm-decode-128k"):
+        out["memory-update:" + name] = measure_memory_update(name, dev, 10, pk)
     return out
 
 
@@ -829,6 +903,10 @@ def main(argv=None):
         torch.cuda.set_device(0)
         dev = torch.device("cuda", 0)
         from retrieval_block_sparse_b200 import synth
+        if args.only_config.startswith("memory-update:"):
+            res = measure_memory_update(args.only_config.split(":", 1)[1], dev, 10, peaks())
+            print(json.dumps({"config": res}), flush=True)
+            return
         w = synth.WORKLOADS[args.only_config]
         fn = measure_decode_config if isinstance(w, synth.DecodeWorkload) else \
             measure_prefill_config

@@ -279,6 +279,62 @@ rba_status rba_stream_step(rba_store* store, const void* q, const void* k_new,
                            float* lse, int32_t* k_used, void* workspace, size_t ws_bytes,
                            cudaStream_t stream);
 
+/* Dynamic memory update ([ML] 2.3.2, dynamic memory update): retrieval
+ * counters decide what the memory keeps once it overflows.  The newest entries
+ * are kept, the oldest are dropped, and from the entries between them the
+ * least retrieved are deleted until the requested number remains.
+ *
+ * Memory unit: the update and its counters are per (batch, kv head) for the
+ * dot-product modes and per batch row for RBA_REP_EMBED_COSINE, whose bank
+ * entry carries the K/V of every kv head.  rba_memory_units() reports the
+ * count U (B * Hkv or B).  Entry = one block (one token when bs = 1).
+ *
+ * Counters: device uint32 [U][cap_blocks], caller-owned, zeroed before first use.
+ * Element j of unit u counts how often block j of that unit has been selected.
+ *
+ * rba_memory_rule (host only): the page's proportions for n entries, with floor:
+ *   keep_newest = n / 10, drop_oldest = n / 10, keep_total = n / 2. */
+rba_status rba_memory_rule(int64_t n_entries, int64_t* keep_newest, int64_t* drop_oldest,
+                           int64_t* keep_total);
+int32_t rba_memory_units(const rba_store* store);  /* U, or -1 for a NULL store */
+
+/* Adds a selection to the counters: every entry j of row r of idx (device int32
+ * [rows][k], laid out [G][U][k] so that row r belongs to unit r % U -- a decode
+ * step's [B][Hkv][k] for dot modes, a prefill's [n_chunks][n_sel][k] with a
+ * batch-1 store, or one row per batch row for the cosine bank) adds one to
+ * counters[r % U][j].  Entries outside [0, cap_blocks) are skipped and flagged
+ * as RBA_ERR_BOUNDS in the status word.  Integer atomics: the result does not
+ * depend on the order.  Errors: INVALID_ARG (rows not a multiple of U), CUDA. */
+rba_status rba_count_retrievals(const rba_store* store, const int32_t* idx, int32_t rows,
+                                int32_t k, uint32_t* counters, cudaStream_t stream);
+
+/* Prunes and compacts the store in place.  The store holds T tokens: full blocks
+ * [0, nb = T / bs) and a partial tail of T - nb * bs tokens.  Blocks [0,
+ * pinned_blocks) (for example attention-sink blocks) are outside the rule and
+ * never move.  The n = nb - pinned_blocks entries after them are updated:
+ *   - the drop_oldest oldest entries are deleted;
+ *   - the keep_newest newest entries are kept;
+ *   - from the entries between them, the least retrieved are deleted (equal
+ *     counts: the older entry first) until keep_total entries remain.
+ * Kept entries stay in order at blocks pinned_blocks, pinned_blocks + 1, ...
+ * Each moves with its K/V rows (every kv head of the unit), its representation,
+ * its positions (RBA_REP_TOPR_ATTN) and its counter.  The tail's tokens follow
+ * the kept blocks.  Counters of the vacated blocks up to the old tail's block
+ * are zeroed.  *T_new (host, may be NULL) receives
+ * (pinned_blocks + keep_total) * bs + tail.
+ *   keep_map  device int32 [U][keep_total], written: keep_map[u][t] = the old index
+ *             of the block now at pinned_blocks + t (may be NULL when keep_total = 0)
+ * Requires 0 <= pinned_blocks <= nb, keep_newest + drop_oldest <= n and
+ * keep_newest <= keep_total <= n - drop_oldest.  Launches one selection kernel,
+ * ceil(keep_total / max(drop_oldest, 1)) move kernels (each moves entries that
+ * are at least drop_oldest blocks from their destination, so no move overwrites
+ * a block that is still to be read), and one kernel for the tail and counters.
+ * Errors: INVALID_ARG, UNSUPPORTED (nb >= 2^31 - 1), CUDA. */
+rba_status rba_memory_update(rba_store* store, int64_t T, int32_t pinned_blocks,
+                             int64_t keep_newest, int64_t drop_oldest, int64_t keep_total,
+                             uint32_t* counters, int32_t* keep_map, int64_t* T_new,
+                             cudaStream_t stream);
+
 /* rba_decode_step from and to host memory: copies q_host (host, dtype [B][Hq][D]) into
  * q_dev, runs the step, copies out/lse/idx back into the host buffers (any of lse_host,
  * idx_host may be NULL), then synchronises `stream`.  q_dev, idx_dev, out_dev, lse_dev are

@@ -9,8 +9,8 @@ All computation is in the CUDA library ``librba.so`` (C ABI:
 ``include/rba.h``); ``rba`` is its Python binding.  ``synth`` draws the seeded
 synthetic inputs.
 """
-from .rba import (Store, RbaError, topk, lib, status_string,  # noqa: F401
+from .rba import (Store, RbaError, topk, memory_rule, lib, status_string,  # noqa: F401
                   OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA,
                   ERR_TIMEOUT, ERR_BOUNDS, LIB_PATH, SIGNATURES)
 
-__all__ = ["Store", "RbaError", "topk", "lib", "status_string", "LIB_PATH", "SIGNATURES"]
+__all__ = ["Store", "RbaError", "topk", "memory_rule", "lib", "status_string", "LIB_PATH", "SIGNATURES"]

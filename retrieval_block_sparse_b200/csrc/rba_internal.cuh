@@ -29,6 +29,7 @@ enum Where : int32_t {
   kWhereMemorize = 4,
   kWherePrefill = 5,
   kWhereFused = 6,
+  kWhereMemory = 7,
 };
 
 __device__ __forceinline__ void report(int32_t* status, int32_t code, int32_t where,

@@ -47,6 +47,12 @@ SIGNATURES = {
     "rba_decode_step_plan": (_c_i32, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
     "rba_stream_step": (_c_i32, [_p, _p, _p, _p, _c_i64, _c_i32, _c_i32, _c_i32, _c_f32, _p,
                                  _c_i32, _p, _p, _p, ctypes.POINTER(_c_i32), _p, _c_size, _p]),
+    "rba_memory_rule": (_c_i32, [_c_i64, ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i64),
+                                 ctypes.POINTER(_c_i64)]),
+    "rba_memory_units": (_c_i32, [_p]),
+    "rba_count_retrievals": (_c_i32, [_p, _p, _c_i32, _c_i32, _p, _p]),
+    "rba_memory_update": (_c_i32, [_p, _c_i64, _c_i32, _c_i64, _c_i64, _c_i64, _p, _p,
+                                   ctypes.POINTER(_c_i64), _p]),
     "rba_decode_step_host": (_c_i32, [_p, _p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32, _p, _p,
                                       _p, _p, _p, _p, _p, _c_size, _p]),
     "rba_store_check": (_c_i32, [_p, _p]),
@@ -306,6 +312,43 @@ class Store:
         sel = idx.reshape(-1)[: self.B * self.Hkv * kk].reshape(self.B, self.Hkv, kk)
         return sel, out, lse
 
+    # -- dynamic memory update ---------------------------------------------------
+    def memory_units(self):
+        """Memory units U: B * Hkv (dot modes) or B (cosine bank)."""
+        return lib().rba_memory_units(self.handle)
+
+    def new_counters(self):
+        """Zeroed retrieval counters [U][cap_blocks] (uint32 in the library; held
+        here as int32 with the same bits)."""
+        return torch.zeros((self.memory_units(), self.cap_blocks), dtype=torch.int32,
+                           device=self.k.device)
+
+    def count_retrievals(self, idx, counters):
+        """Adds the selection idx ([..., U, k] int32, row r -> unit r % U) to counters."""
+        k = idx.shape[-1]
+        rows = idx.numel() // k if k else 0
+        _check(lib().rba_count_retrievals(self.handle, _ptr(idx), rows, k, _ptr(counters),
+                                          _stream()), "rba_count_retrievals")
+
+    def memory_update(self, T, counters, *, pinned_blocks=0, keep_newest=None, drop_oldest=None,
+                      keep_total=None, keep_map=None):
+        """Counter-driven prune and in-place compaction of the T tokens held.
+        Counts not given follow memory_rule(n) for the n = T // bs - pinned_blocks
+        entries.  Returns (T_new, keep_map [U][keep_total])."""
+        n = T // self.bs - pinned_blocks
+        rule = memory_rule(max(n, 0))
+        keep_newest = rule[0] if keep_newest is None else keep_newest
+        drop_oldest = rule[1] if drop_oldest is None else drop_oldest
+        keep_total = rule[2] if keep_total is None else keep_total
+        if keep_map is None:
+            keep_map = torch.empty((self.memory_units(), max(keep_total, 1)), dtype=torch.int32,
+                                   device=self.k.device)
+        t_new = _c_i64(0)
+        _check(lib().rba_memory_update(self.handle, T, pinned_blocks, keep_newest, drop_oldest,
+                                       keep_total, _ptr(counters), _ptr(keep_map),
+                                       ctypes.byref(t_new), _stream()), "rba_memory_update")
+        return t_new.value, keep_map[:, :keep_total]
+
     def decode_step_host(self, q_host, k, T, sink, window, *, q_dev, idx_dev, out_dev, lse_dev,
                          out_host, lse_host=None, idx_host=None, workspace, scale=None):
         """Host buffers in and out; synchronises the current stream."""
@@ -321,6 +364,14 @@ class Store:
     def check(self):
         """Synchronises and raises if a kernel recorded a device-side error."""
         _check(lib().rba_store_check(self.handle, _stream()), "device status")
+
+
+def memory_rule(n):
+    """(keep_newest, drop_oldest, keep_total) for n memory entries (host only)."""
+    a, b, c = _c_i64(), _c_i64(), _c_i64()
+    _check(lib().rba_memory_rule(n, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "rba_memory_rule")
+    return a.value, b.value, c.value
 
 
 def topk(scores, k, *, index_base=0, out=None, workspace=None):

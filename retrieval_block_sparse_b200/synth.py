@@ -140,7 +140,7 @@ WORKLOADS = {
 
 _TENSOR_IDS = {"K": 1, "V": 2, "q": 3, "probe": 4, "landmarks": 5, "u": 6,
                "planted": 7, "bank_embed": 8, "query_embed": 9, "Q": 10,
-               "chunk_K": 11, "chunk_V": 12, "pick": 13, "scores": 14}
+               "chunk_K": 11, "chunk_V": 12, "pick": 13, "scores": 14, "counts": 15}
 
 
 def _stream(seed: int, tensor: str, index: int = 0) -> np.random.Generator:
@@ -324,3 +324,22 @@ def random_scores(seed: int, rows: int, n: int, ties: int = 0) -> np.ndarray:
         lv = np.sort(_normal(seed + 1, "scores", (1, ties))[0])
         x = lv[np.floor((x - x.min()) / (x.max() - x.min() + 1e-9) * ties).astype(np.int64).clip(0, ties - 1)]
     return np.ascontiguousarray(x, dtype=np.float32)
+
+
+# ---------------------------------------------------------------------------
+# retrieval counters (for the dynamic memory update)
+
+
+def retrieval_counts(seed: int, units: int, n: int, huge: float = 0.0) -> np.ndarray:
+    """uint32 retrieval-frequency counters [units][n]: most entries rarely
+    retrieved (Poisson mean 0.7), about 30% often (Poisson mean 20), so equal
+    counts are frequent.  A fraction ``huge`` of the entries gets a count in
+    [2^31, 2^32) (exercises every byte of a 32-bit count)."""
+    g = _stream(seed, "counts")
+    c = g.poisson(0.7, size=(units, n)).astype(np.uint64)
+    hot = g.random((units, n)) < 0.3
+    c[hot] = g.poisson(20.0, size=int(hot.sum()))
+    if huge > 0:
+        big = g.random((units, n)) < huge
+        c[big] = g.integers(1 << 31, (1 << 32) - 1, size=int(big.sum()))
+    return c.astype(np.uint32)

@@ -127,3 +127,42 @@ def test_workspace_sizes_are_positive(L):
     assert L.rba_topk_workspace_size(8, 1 << 20, 2048) > 8 * (1 << 20) * 8
     assert L.rba_topk_workspace_size(8, 1000, 32) == 0
     L.rba_store_destroy(h)
+
+
+def test_memory_rule_matches_oracle(L):
+    a, b, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    for n in list(range(0, 64)) + [99, 100, 101, 7936, 1 << 20, (1 << 31) - 3]:
+        assert L.rba_memory_rule(n, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == 0
+        assert (a.value, b.value, c.value) == O.memory_rule(n)
+    assert L.rba_memory_rule(-1, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == 1
+
+
+def test_memory_units_per_mode(L):
+    s, h = _create(L, batch=3, n_kv_heads=2, n_q_heads=4)
+    assert L.rba_memory_units(h) == 6
+    L.rba_store_destroy(h)
+    s, h = _create(L, batch=3, n_kv_heads=2, n_q_heads=4, mode=3, d_ret=32)
+    assert L.rba_memory_units(h) == 3                     # the cosine bank is per batch row
+    L.rba_store_destroy(h)
+    assert L.rba_memory_units(None) == -1
+
+
+def test_memory_update_argument_checks_launch_nothing(L):
+    s, h = _create(L, block_size=16, capacity_tokens=1024)  # U = 2, cap_blocks = 64
+    i64 = ctypes.c_int64
+    T = 40 * 16 + 5                                         # nb = 40, tail 5
+    upd = lambda T, pin, nw, od, kt, cnt=FAKE, km=FAKE: L.rba_memory_update(  # noqa: E731
+        h, i64(T), pin, i64(nw), i64(od), i64(kt), cnt, km, None, None)
+    assert upd(T, 0, 4, 4, 37) == 1                         # keep_total > n - drop_oldest
+    assert upd(T, 0, 4, 4, 3) == 1                          # keep_total < keep_newest
+    assert upd(T, 0, 30, 11, 30) == 1                       # newest + oldest > n
+    assert upd(T, 41, 0, 0, 0) == 1                         # pinned beyond the full blocks
+    assert upd(2000, 0, 0, 0, 0) == 1                       # T above the capacity
+    assert upd(T, 0, 4, 4, 20, cnt=None) == 1               # no counters
+    assert upd(T, 0, 4, 4, 20, km=None) == 1                # no keep map
+    assert upd(T, -1, 4, 4, 20) == 1
+    # counting: rows must be a whole number of units; an empty selection is a no-op
+    assert L.rba_count_retrievals(h, FAKE, 3, 4, FAKE, None) == 1
+    assert L.rba_count_retrievals(h, FAKE, 2, 0, FAKE, None) == 0
+    assert L.rba_count_retrievals(h, FAKE, 2, 4, None, None) == 1
+    L.rba_store_destroy(h)
