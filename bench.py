@@ -48,6 +48,8 @@ KERNEL_SOURCES = {
     "attend_decode_kernel": ["csrc/attend.cu", "csrc/attend_impl.cuh", "csrc/rba_internal.cuh"],
     "decode_fused_kernel": ["csrc/decode_fused.cu", "csrc/attend_impl.cuh",
                             "csrc/rba_internal.cuh"],
+    "decode_mma_kernel": ["csrc/decode_fused.cu", "csrc/attend_impl.cuh",
+                          "csrc/rba_internal.cuh", "csrc/tmap.cu"],
 }
 
 
@@ -425,7 +427,7 @@ def run_ours(args):
     att_gbs = gath_b / (att_us * 1e-6) / 1e9
     step_us = ms_max * 1e3 / args.steps
     step_gbs = bytes_step / (step_us * 1e-6) / 1e9
-    dom = "decode_fused_kernel" if plan == 1 else "attend_decode_kernel"
+    dom = {1: "decode_fused_kernel", 2: "decode_mma_kernel"}.get(plan, "attend_decode_kernel")
     dom_bytes, dom_us, dom_gbs = gath_b, att_us, att_gbs
     traffic = traffic_lookup(dom, args.workload)
 
@@ -507,8 +509,9 @@ def run_ours(args):
         "gpu_launches": launches * args.steps,
         "kernels_per_step": launches,
         "graph_kernel_nodes_per_step": n_nodes,
-        "path": ("score -> top-k -> persistent attention (programmatic dependent launches)"
-                 if plan == 1 else f"score -> top-k -> split-K attention (plan {plan})"),
+        "path": ("score -> top-k -> persistent attention (programmatic dependent launches; "
+                 + ("whole-block tensor-core kernel)" if plan == 2 else "CUDA-core kernel)")
+                 if plan in (1, 2) else f"score -> top-k -> split-K attention (plan {plan})"),
         "cpu_baseline": cpu,
         "configs": configs,
     }
@@ -633,7 +636,9 @@ def measure_decode_config(name, dev, seconds, pk):
     return {"workload": name, "steps_per_s": round(1e6 / us, 2), "us_per_step": round(us, 3),
             "algorithmic_bytes": nbytes, "rep_key_bytes": rep_b, "gathered_kv_bytes": gath_b,
             "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
-            "path": "pipelined, persistent attention" if plan == 1 else "split-K attention",
+            "path": {1: "pipelined, persistent attention (CUDA cores)",
+                     2: "pipelined, persistent attention (whole-block, tensor cores)"}.get(
+                         plan, "split-K attention"),
             "steps_timed": n * len(stores),
             "l2": (f"L2-sized write between steps, its time subtracted" if use_flush else
                    f"{len(stores)} store replicas rotated ({len(stores)} x {nbytes / 1e6:.1f} MB"

@@ -167,7 +167,7 @@ size_t rba_topk_workspace_size(int32_t rows, int32_t n, int32_t k);
  * states ([IL] overall framework: local window + a few memory units; [ML]
  * 2.3.3 retrieved chunks attended without a causal mask).  Runs the
  * persistent attention kernel (one CTA per SM, bulk-copy staging) where
- * rba_decode_step_plan() would report 1, else a split-K kernel.
+ * rba_decode_step_plan() would report 1 or 2, else a split-K kernel.
  *   q    device dtype [B][Hq][D];  idx device int32 [B][Hkv][k] ascending candidate block ids
  *   out  device fp32 [B][Hq][D];   lse device fp32 [B][Hq] (natural log) or NULL
  *   For q head i of kv head h = i / (Hq/Hkv):
@@ -231,7 +231,7 @@ size_t rba_attend_prefill_workspace_size(const rba_store* store, int32_t n_chunk
 
 /* One whole decode step: rba_score (dot modes) -> rba_topk per (b, kv head)
  * -> rba_attend, with the same definitions as those calls, as three kernels
- * on `stream`.  Where rba_decode_step_plan() reports 1, the top-k kernel and
+ * on `stream`.  Where rba_decode_step_plan() reports 1 or 2, the top-k kernel and
  * the persistent attention kernel are programmatic dependents of the kernel
  * before them: they start early, the attention kernel streams the sink and
  * window rows, and each waits on the device for its inputs.
@@ -248,8 +248,11 @@ size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t
                                       int32_t sink, int32_t window);
 
 /* How rba_decode_step runs this problem (host only; queries the device, launches nothing):
- *   1   score -> top-k -> persistent attention kernel, the last two as programmatic
- *       dependents (overlapped); k <= 2048, GQA group of 1, 2 or 4
+ *   2   score -> top-k -> persistent attention kernel, the last two as programmatic
+ *       dependents (overlapped); the attention kernel is the whole-block one: bf16 store,
+ *       block size a multiple of 64, head dim 64 or 128; inner products on tensor cores
+ *   1   as 2 with the CUDA-core attention kernel (other block sizes, fp32); k <= 2048,
+ *       GQA group of 1, 2 or 4 in both
  *   0   score -> top-k -> split-K attention, in stream order: outside those limits
  *  -2   within the limits but no CTA of the persistent kernel fits on an SM (as 0)
  *  -3   a CUDA error while asking (as 0)

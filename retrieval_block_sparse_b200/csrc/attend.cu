@@ -342,7 +342,7 @@ int32_t rba_decode_step_plan(const rba_store* st, int32_t k, int64_t T, int32_t 
   const int occ = fused_occupancy(st);
   if (occ < 0) return -3;
   if (occ == 0) return -2;
-  return 1;
+  return fused_whole_blocks(st) ? 2 : 1;
 }
 
 size_t rba_decode_step_workspace_size(const rba_store* st, int32_t k, int64_t T, int32_t sink,

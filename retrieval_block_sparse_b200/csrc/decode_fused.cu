@@ -151,9 +151,10 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
                : "memory");
   return old;
 }
-// barrier of the compute warps only (warp 0 never joins it)
+// barrier of the NCT compute threads only (warp 0 never joins it)
+template <int NCT>
 __device__ __forceinline__ void compute_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(NCT) : "memory");
 }
 __device__ __forceinline__ int ctid() { return static_cast<int>(threadIdx.x) - 32; }
 
@@ -233,10 +234,46 @@ __device__ __forceinline__ bool next_item(const FusedArgs& a, Iter& it, Item& ou
 // ---------------------------------------------------------------------------
 // shared memory layout
 
+// Stage geometry: a stage holds TT rows of K then TT rows of V; rows are ROWB
+// bytes long and RSTR bytes apart.  RSTR == ROWB: a contiguous run of rows is
+// one bulk copy; RSTR > ROWB (padded rows): one bulk copy per row.
+template <int TT_, int ROWB_, int RSTR_>
+struct StageGeo {
+  static constexpr int TT = TT_, ROWB = ROWB_, RSTR = RSTR_;
+  static constexpr int VOFF = TT * RSTR;
+  static constexpr int STAGE = 2 * TT * RSTR;
+  static_assert(RSTR % 16 == 0 && ROWB % 16 == 0, "bulk copies move 16-byte multiples");
+};
+
 struct __align__(16) Meta {
   int nrows;
   int pad[3];
 };
+
+// Small shared variables after the stage ring, the warp states and the
+// selection layout (MISC bytes): full[kMaxStages], empty[kMaxStages] (mbarriers),
+// meta[kMaxStages], then ints: [0..16) flags, [16..20) abort flag, [20..148)
+// floats (merge factors and maxima), [148..150) the merge mbarrier.
+struct MiscLayout {
+  uint64_t* full;
+  uint64_t* empty;
+  Meta* meta;
+  int* s_misc;
+  volatile int* abort_flag;
+  float* s_f;         // [128]: fac [G * NW] (<= 112), gmax [G] at +112
+  uint64_t* merge_bar;
+  __device__ explicit MiscLayout(char* misc) {
+    full = reinterpret_cast<uint64_t*>(misc);
+    empty = full + kMaxStages;
+    meta = reinterpret_cast<Meta*>(empty + kMaxStages);
+    s_misc = reinterpret_cast<int*>(meta + kMaxStages);
+    abort_flag = s_misc + 16;
+    s_f = reinterpret_cast<float*>(s_misc + 20);
+    merge_bar = reinterpret_cast<uint64_t*>(s_misc + 148);
+  }
+};
+constexpr int kMiscBytes = 1024;
+static_assert(2 * kMaxStages * 8 + kMaxStages * 16 + 150 * 4 <= kMiscBytes, "misc layout");
 
 template <typename T, int D, int G>
 struct FusedSmem {
@@ -246,9 +283,144 @@ struct FusedSmem {
   // regions after the stage ring (NS * STAGE, chosen at launch)
   static constexpr int RED = up16(kCW * G * (D + 2) * 4);       // warp states
   static constexpr int SEL = (kMaxK + 4) * 4 * 2;               // selected prefix + starts
-  static constexpr int MISC = 1024;
+  static constexpr int MISC = kMiscBytes;
   static size_t bytes(int NS) { return size_t(NS) * STAGE + RED + SEL + MISC; }
 };
+
+// ---------------------------------------------------------------------------
+// end of a head: NW per-warp states -> output, or -> a partial slot and the
+// last part's merge
+
+// red[w][g] = (m, l, o[D]) of warp w (log2 units, o unnormalised).  Combines
+// the NW states of head bh held by this CTA; with m == 1 writes out and lse,
+// else publishes the state to slot `ord` of the head and, if this CTA is the
+// head's last part to finish (acq_rel ticket), merges the head's m slots,
+// which arrive by bulk copies into the (idle) stage ring.  Called by all NCT
+// compute threads; ends with them synchronised.
+template <int G, int D, int NW, int NCT>
+__device__ __forceinline__ void finish_head(const FusedArgs& a, int bh, int ord, const float* red,
+                            const MiscLayout& ms, char* stages, size_t ring_bytes,
+                            uint32_t& merge_ph) {
+  constexpr int kSlotFloats = slot_floats(G, D);
+  static_assert(G * NW <= 112 && G <= 16, "merge factors fit the misc floats");
+  const int tid = ctid();
+  float* fac = ms.s_f;          // [G][NW] factors exp2(m_w - M) of the NW warp states
+  float* gmax = ms.s_f + 112;   // [G] the max M
+  compute_sync<NCT>();
+  if (tid < G * NW) {
+    const int gg = tid / NW, w = tid % NW;
+    float M = -INFINITY;
+    for (int v = 0; v < NW; ++v) M = fmaxf(M, red[(v * G + gg) * (D + 2)]);
+    const float mw = red[(w * G + gg) * (D + 2)];
+    fac[tid] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+    if (w == 0) gmax[gg] = M;
+  }
+  compute_sync<NCT>();
+  const int b = bh / a.at.Hkv, h = bh % a.at.Hkv;
+  if (a.m == 1) {
+    // this CTA holds the whole head
+    for (int x = tid; x < G * D; x += NCT) {
+      const int gg = x / D, d = x % D;
+      float num = 0.f, den = 0.f;
+      for (int w = 0; w < NW; ++w) {
+        const float f = fac[gg * NW + w];
+        num += red[(w * G + gg) * (D + 2) + 2 + d] * f;
+        den += red[(w * G + gg) * (D + 2) + 1] * f;
+      }
+      a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = den > 0.f ? num / den : 0.f;
+      if (d == 0 && a.at.lse != nullptr)
+        a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
+            den > 0.f ? (gmax[gg] + log2f(den)) * 0.6931471805599453f : -INFINITY;
+    }
+  } else {
+    // this CTA's state -> slot `ord` of the head; the last of the head's m
+    // parts to finish merges all m slots
+    const bool slot_ok = ord >= 0 && ord < a.m;
+    if (!slot_ok && tid == 0) report(a.at.status, RBA_ERR_BOUNDS, kWhereFused, 4);
+    float* base = a.slots + int64_t(bh) * a.m * kSlotFloats;
+    float* slot = base + int64_t(slot_ok ? ord : 0) * kSlotFloats;
+#pragma unroll 1
+    for (int x = tid; x < G * (D + 2) && slot_ok; x += NCT) {
+      const int gg = x / (D + 2), c = x % (D + 2);
+      float acc = 0.f;
+      if (c == 0) {
+        acc = gmax[gg];
+      } else {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) acc += red[(w * G + gg) * (D + 2) + c] * fac[gg * NW + w];
+      }
+      slot[x] = acc;
+    }
+    compute_sync<NCT>();
+    if (tid == 0) {
+      const uint32_t t = atom_add_acq_rel(a.tickets + bh, 1u);  // publishes our slot
+      ms.s_misc[9] = t == uint32_t(a.m - 1);
+    }
+    compute_sync<NCT>();
+    if (ms.s_misc[9]) {
+      // the last part of the head merges the m slots.  The slots go to shared
+      // memory by bulk copies into the stage ring (idle: with m > 1 a CTA
+      // holds one part of one head, all of it consumed), a chunk at a time;
+      // each thread then folds every slot's (m, l, o[d]) of its output
+      // elements (g, d) into a running (max, sum, output).
+      constexpr int SLOT = kSlotFloats * 4;  // a multiple of 16 bytes
+      constexpr int NX = (G * D + NCT - 1) / NCT;
+      const int nl = a.m;
+      const int chunk = static_cast<int>(ring_bytes / SLOT);
+      float M[NX], L[NX], O[NX];
+#pragma unroll
+      for (int r = 0; r < NX; ++r) {
+        M[r] = -INFINITY;
+        L[r] = 0.f;
+        O[r] = 0.f;
+      }
+      for (int j0 = 0; j0 < nl; j0 += chunk) {
+        const int n = min(chunk, nl - j0);
+        if (tid == 0) {
+          // (the compute warps' reads of the ring are ordered before the copies)
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_arrive_tx(ms.merge_bar, uint32_t(n) * SLOT);
+          for (int j = 0; j < n; ++j)
+            bulk_g2s(stages + size_t(j) * SLOT, base + int64_t(j0 + j) * kSlotFloats, SLOT,
+                     ms.merge_bar);
+        }
+        const bool ok = mbar_wait(ms.merge_bar, merge_ph, ms.abort_flag, a.at.status, 6);
+        if (!ok && tid == 0) mbar_drain(ms.merge_bar, merge_ph);  // no copy outlives the CTA
+        merge_ph ^= 1u;
+        const float* sm = reinterpret_cast<const float*>(stages);
+#pragma unroll
+        for (int r = 0; r < NX; ++r) {
+          const int x = tid + r * NCT;
+          if (!ok || x >= G * D) continue;
+          const int gg = x / D, d = x % D;
+          for (int j = 0; j < n; ++j) {
+            const float* q = sm + j * kSlotFloats + gg * (D + 2);
+            const float mj = q[0], lj = q[1], oj = q[2 + d];
+            const float mn = fmaxf(M[r], mj);
+            const float sa = M[r] == -INFINITY ? 0.f : exp2f(M[r] - mn);
+            const float sb = mj == -INFINITY ? 0.f : exp2f(mj - mn);
+            L[r] = L[r] * sa + lj * sb;
+            O[r] = O[r] * sa + oj * sb;
+            M[r] = mn;
+          }
+        }
+        compute_sync<NCT>();  // the chunk buffer is read before the next copy
+      }
+#pragma unroll
+      for (int r = 0; r < NX; ++r) {
+        const int x = tid + r * NCT;
+        if (x >= G * D) continue;
+        const int gg = x / D, d = x % D;
+        a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = L[r] > 0.f ? O[r] / L[r] : 0.f;
+        if (d == 0 && a.at.lse != nullptr)
+          a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
+              L[r] > 0.f ? (M[r] + log2f(L[r])) * 0.6931471805599453f : -INFINITY;
+      }
+      if (tid == 0) a.tickets[bh] = 0;  // zero again for the next call
+    }
+  }
+  compute_sync<NCT>();
+}
 
 // LaneState query slice from a [G][D] fp32 copy in shared memory (the same
 // values and lane layout as load_q).
@@ -282,10 +454,9 @@ __device__ __forceinline__ void load_q_smem(const float* qs, float scale_log2,
 // Stages one item into `stg`: bulk copies that complete on `bar`, whose
 // transaction count is armed with the item's bytes.  Selected rows need the
 // selection, which the caller has waited for.
-template <typename T, int D, int RW>
+template <class Geo>
 __device__ void issue_item(const FusedArgs& a, const Item& item, char* stg, uint64_t* bar,
                            Meta* meta, int* sel_pref, int* sel_phys, int* sel_bh) {
-  using C = DecodeTile<T, D, RW>;
   const int lane = threadIdx.x & 31;
   const int* pref;
   const int* phys;
@@ -343,7 +514,7 @@ __device__ void issue_item(const FusedArgs& a, const Item& item, char* stg, uint
   const int nrows = v1 > v0 ? v1 - v0 : 0;
   if (lane == 0) {
     meta->nrows = nrows;
-    mbar_arrive_tx(bar, uint32_t(nrows) * C::ROWB * 2);
+    mbar_arrive_tx(bar, uint32_t(nrows) * Geo::ROWB * 2);
   }
   __syncwarp();
   if (nrows > 0) {
@@ -355,25 +526,41 @@ __device__ void issue_item(const FusedArgs& a, const Item& item, char* stg, uint
     }
     const char* Kb = static_cast<const char*>(a.at.K);
     const char* Vb = static_cast<const char*>(a.at.V);
-    for (int sg = lo + lane; sg < nseg && pref[sg] < v1; sg += 32) {
-      const int a0 = max(v0, pref[sg]), a1 = min(v1, pref[sg + 1]);
-      if (a1 <= a0) continue;
-      const int64_t tok = int64_t(item.bh) * a.at.cap + phys[sg] + (a0 - pref[sg]);
-      const uint32_t bytes = uint32_t(a1 - a0) * C::ROWB;
-      const int row = a0 - v0;
-      bulk_g2s(stg + row * C::ROWB, Kb + tok * C::ROWB, bytes, bar);
-      bulk_g2s(stg + C::TT * C::ROWB + row * C::ROWB, Vb + tok * C::ROWB, bytes, bar);
+    if constexpr (Geo::RSTR == Geo::ROWB) {
+      // one copy per contiguous run (a lane per segment)
+      for (int sg = lo + lane; sg < nseg && pref[sg] < v1; sg += 32) {
+        const int a0 = max(v0, pref[sg]), a1 = min(v1, pref[sg + 1]);
+        if (a1 <= a0) continue;
+        const int64_t tok = int64_t(item.bh) * a.at.cap + phys[sg] + (a0 - pref[sg]);
+        const uint32_t bytes = uint32_t(a1 - a0) * Geo::ROWB;
+        const int row = a0 - v0;
+        bulk_g2s(stg + row * Geo::RSTR, Kb + tok * Geo::ROWB, bytes, bar);
+        bulk_g2s(stg + Geo::VOFF + row * Geo::RSTR, Vb + tok * Geo::ROWB, bytes, bar);
+      }
+    } else {
+      // padded rows: one copy per row (a lane per row); the row's segment is
+      // the last one starting at or before it
+      for (int row = lane; row < nrows; row += 32) {
+        const int v = v0 + row;
+        int l2 = lo, h2 = nseg - 1;
+        while (l2 < h2) {
+          const int mid = (l2 + h2 + 1) >> 1;
+          if (pref[mid] <= v) l2 = mid; else h2 = mid - 1;
+        }
+        const int64_t tok = int64_t(item.bh) * a.at.cap + phys[l2] + (v - pref[l2]);
+        bulk_g2s(stg + row * Geo::RSTR, Kb + tok * Geo::ROWB, Geo::ROWB, bar);
+        bulk_g2s(stg + Geo::VOFF + row * Geo::RSTR, Vb + tok * Geo::ROWB, Geo::ROWB, bar);
+      }
     }
   }
   __syncwarp();
 }
 
 // Warp 0: stage every item of this CTA, in order, into the stage ring.
-template <typename T, int D, int RW>
+template <class Geo>
 __device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64_t* full,
                                         uint64_t* empty, Meta* meta, int* sel_pref,
                                         int* sel_phys, volatile int* abort_flag) {
-  using C = DecodeTile<T, D, RW>;
   const int NS = a.NS;
   Iter it;
   iter_begin(a, it);
@@ -381,7 +568,7 @@ __device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64
   int j = 0, s = 0, sel_bh = -1;
   uint32_t ph = 0;  // phase parity of the stage's next fill
   bool selection_visible = false;
-  while (next_item<C::TT>(a, it, item)) {
+  while (next_item<Geo::TT>(a, it, item)) {
     // stage s is free once every compute warp released its previous item
     if (j >= NS && !mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.at.status, 1)) break;
     if (item.kind == 2 && !selection_visible) {
@@ -390,8 +577,8 @@ __device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64
       asm volatile("griddepcontrol.wait;" ::: "memory");
       selection_visible = true;
     }
-    issue_item<T, D, RW>(a, item, stages + size_t(s) * C::STAGE, &full[s], &meta[s], sel_pref,
-                     sel_phys, &sel_bh);
+    issue_item<Geo>(a, item, stages + size_t(s) * Geo::STAGE, &full[s], &meta[s], sel_pref,
+                    sel_phys, &sel_bh);
     ++j;
     if (++s == NS) {
       s = 0;
@@ -421,13 +608,12 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   int* sel_pref = reinterpret_cast<int*>(reinterpret_cast<char*>(red) + S::RED);
   int* sel_phys = sel_pref + (kMaxK + 1);
   char* misc = reinterpret_cast<char*>(sel_pref) + S::SEL;
-  uint64_t* full = reinterpret_cast<uint64_t*>(misc);               // [kMaxStages]
-  uint64_t* empty = full + kMaxStages;                              // [kMaxStages]
-  Meta* meta = reinterpret_cast<Meta*>(empty + kMaxStages);         // [kMaxStages]
-  int* s_misc = reinterpret_cast<int*>(meta + kMaxStages);          // [16]
-  volatile int* abort_flag = s_misc + 16;                           // [4]
-  uint64_t* merge_bar = reinterpret_cast<uint64_t*>(s_misc + 84);   // [1] (s_f is [64] at +20)
-  float* s_f = reinterpret_cast<float*>(s_misc + 20);               // [64]
+  const MiscLayout ms(misc);
+  uint64_t* full = ms.full;
+  uint64_t* empty = ms.empty;
+  Meta* meta = ms.meta;
+  volatile int* abort_flag = ms.abort_flag;
+  uint64_t* merge_bar = ms.merge_bar;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
@@ -442,7 +628,8 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   }
   __syncthreads();
   if (warp == 0) {
-    produce<T, D, RW>(a, stages, full, empty, meta, sel_pref, sel_phys, abort_flag);
+    produce<StageGeo<C::TT, C::ROWB, C::ROWB>>(a, stages, full, empty, meta, sel_pref, sel_phys,
+                                               abort_flag);
     return;
   }
   // ---- compute warps from here on (named barrier 1; no __syncthreads)
@@ -475,7 +662,7 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
     const T* qp = static_cast<const T*>(a.at.q) + (int64_t(b) * a.at.Hq + h * G) * D;
     for (int x = tid; x < G * D; x += kCT) q_first[x] = Elem<T>::to_f32(qp[x]);
   }
-  compute_sync();
+  compute_sync<kCT>();
 
   Item item;
   bool have = next_item<C::TT>(a, it, item);
@@ -485,36 +672,6 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   int cur_bh = -1;
   int ord = 0;  // part index of head cur_bh held by this CTA (its slot)
   uint32_t merge_ph = 0;  // phase parity of merge_bar
-  float* fac = s_f;         // [G][nw] factors exp2(m_w - M) of the nw warp states
-  float* gmax = s_f + 60;   // [G] the max M
-  // fac / gmax from nw per-warp states red[w][g][m, l, o[D]]
-  auto combine = [&](int nw) {
-    if (tid < G * nw) {
-      const int gg = tid / nw, w = tid % nw;
-      float M = -INFINITY;
-      for (int v = 0; v < nw; ++v) M = fmaxf(M, red[(v * G + gg) * (D + 2)]);
-      const float mw = red[(w * G + gg) * (D + 2)];
-      fac[tid] = mw == -INFINITY ? 0.f : exp2f(mw - M);
-      if (w == 0) gmax[gg] = M;
-    }
-  };
-  // output (and lse) of head cur_bh from nw warp states combined by fac
-  auto write_out = [&](int nw) {
-    const int b = cur_bh / a.at.Hkv, h = cur_bh % a.at.Hkv;
-    for (int x = tid; x < G * D; x += kCT) {
-      const int gg = x / D, d = x % D;
-      float num = 0.f, den = 0.f;
-      for (int w = 0; w < nw; ++w) {
-        const float f = fac[gg * nw + w];
-        num += red[(w * G + gg) * (D + 2) + 2 + d] * f;
-        den += red[(w * G + gg) * (D + 2) + 1] * f;
-      }
-      a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = den > 0.f ? num / den : 0.f;
-      if (d == 0 && a.at.lse != nullptr)
-        a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
-            den > 0.f ? (gmax[gg] + log2f(den)) * 0.6931471805599453f : -INFINITY;
-    }
-  };
   while (true) {
     const bool more = have;
     if (cur_bh >= 0 && (!more || item.bh != cur_bh)) {
@@ -542,100 +699,8 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
           }
         }
       }
-      compute_sync();
-      combine(RW);
-      compute_sync();
-      if (a.m == 1) {
-        write_out(RW);  // this CTA holds the whole head
-      } else {
-        // this CTA's state -> slot `ord` of the head; the last of the head's
-        // m parts to finish merges all m slots
-        const bool slot_ok = ord >= 0 && ord < a.m;
-        if (!slot_ok && tid == 0) report(a.at.status, RBA_ERR_BOUNDS, kWhereFused, 4);
-        float* base = a.slots + int64_t(cur_bh) * a.m * kSlotFloats;
-        float* slot = base + int64_t(slot_ok ? ord : 0) * kSlotFloats;
-#pragma unroll 1
-        for (int x = tid; x < G * (D + 2) && slot_ok; x += kCT) {
-          const int gg = x / (D + 2), c = x % (D + 2);
-          float acc = 0.f;
-          if (c == 0) {
-            acc = gmax[gg];
-          } else {
-#pragma unroll
-            for (int w = 0; w < RW; ++w)
-              acc += red[(w * G + gg) * (D + 2) + c] * fac[gg * RW + w];
-          }
-          slot[x] = acc;
-        }
-        compute_sync();
-        if (tid == 0) {
-          const uint32_t t = atom_add_acq_rel(a.tickets + cur_bh, 1u);  // publishes our slot
-          s_misc[9] = t == uint32_t(a.m - 1);
-        }
-        compute_sync();
-        if (s_misc[9]) {
-          // the last part of the head merges the m slots.  The slots go to
-          // shared memory by bulk copies into the stage ring (idle: with
-          // m > 1 a CTA holds one part of one head, all of it consumed), a
-          // chunk at a time; each thread then folds every slot's (m, l, o[d])
-          // of its output elements (g, d) into a running (max, sum, output).
-          constexpr int SLOT = kSlotFloats * 4;  // a multiple of 16 bytes
-          const int nl = a.m;
-          const int chunk = (NS * C::STAGE) / SLOT;
-          const int b = cur_bh / a.at.Hkv, h = cur_bh % a.at.Hkv;
-          float M[2], L[2], O[2];  // elements x = tid and tid + kCT
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            M[r] = -INFINITY;
-            L[r] = 0.f;
-            O[r] = 0.f;
-          }
-          for (int j0 = 0; j0 < nl; j0 += chunk) {
-            const int n = min(chunk, nl - j0);
-            if (tid == 0) {
-              // (the compute warps' reads of the ring are ordered before the copies)
-              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-              mbar_arrive_tx(merge_bar, uint32_t(n) * SLOT);
-              for (int j = 0; j < n; ++j)
-                bulk_g2s(stages + size_t(j) * SLOT, base + int64_t(j0 + j) * kSlotFloats, SLOT,
-                         merge_bar);
-            }
-            const bool ok = mbar_wait(merge_bar, merge_ph, abort_flag, a.at.status, 6);
-            if (!ok && tid == 0) mbar_drain(merge_bar, merge_ph);  // no copy outlives the CTA
-            merge_ph ^= 1u;
-            const float* sm = reinterpret_cast<const float*>(stages);
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int x = tid + r * kCT;
-              if (!ok || x >= G * D) continue;
-              const int gg = x / D, d = x % D;
-              for (int j = 0; j < n; ++j) {
-                const float* q = sm + j * kSlotFloats + gg * (D + 2);
-                const float mj = q[0], lj = q[1], oj = q[2 + d];
-                const float mn = fmaxf(M[r], mj);
-                const float sa = M[r] == -INFINITY ? 0.f : exp2f(M[r] - mn);
-                const float sb = mj == -INFINITY ? 0.f : exp2f(mj - mn);
-                L[r] = L[r] * sa + lj * sb;
-                O[r] = O[r] * sa + oj * sb;
-                M[r] = mn;
-              }
-            }
-            compute_sync();  // the chunk buffer is read before the next copy
-          }
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int x = tid + r * kCT;
-            if (x >= G * D) continue;
-            const int gg = x / D, d = x % D;
-            a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = L[r] > 0.f ? O[r] / L[r] : 0.f;
-            if (d == 0 && a.at.lse != nullptr)
-              a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
-                  L[r] > 0.f ? (M[r] + log2f(L[r])) * 0.6931471805599453f : -INFINITY;
-          }
-          if (tid == 0) a.tickets[cur_bh] = 0;  // zero again for the next call
-        }
-      }
-      compute_sync();
+      finish_head<G, D, RW, kCT>(a, cur_bh, ord, red, ms, stages, size_t(NS) * C::STAGE,
+                                 merge_ph);
       cur_bh = -1;
     }
     if (!more) break;
@@ -656,34 +721,521 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(FusedArgs a) {
   }
 }
 
-constexpr size_t kMaxSmem = 227 * 1024;  // dynamic shared memory of one CTA
+// ---------------------------------------------------------------------------
+// bf16 with whole-block tiles: the inner products on the tensor cores
+//
+// Used when every retrieved block is a whole number of 64-row tiles.  The
+// staging warp cuts the CTA's rows into pieces that never cross a segment
+// (sink, window, one selected block) and are at most 64 rows long, and loads
+// each piece as 64-row boxes of K and V (two 64-column halves each) with 2-D
+// bulk tensor copies in the 128-byte swizzled layout; rows of a box past the
+// piece are ignored.  It records each piece's head, part and row count in the
+// stage's meta word, which drives the compute warps.
+//
+// Per warp and 16-row slice of a tile (mma.sync m16n8k16, bf16 in, fp32
+// accumulate), with the q heads of the kv head padded to M = 16:
+//   S^T[16][16 rows]  = Q[16][D] . K^T           (D/16 k-steps, 2 n-tiles of 8 rows)
+//   online softmax per head over the rows (a lane holds 4 rows of head lane/4)
+//   O[16][D]         += P^T[16][16 rows] . V     (D/8 n-tiles, one k-step)
+// P^T comes straight from the S^T accumulators (the C layout of two 8-row
+// n-tiles is the A layout of one 16-row k-step).  P is split as p = hi + lo,
+// both bf16, and multiplied twice, so the weights keep ~16 mantissa bits.
+// K and V fragments come from shared memory by ldmatrix (V transposed); the
+// swizzle puts the eight rows of a matrix in distinct banks.
 
-template <typename T, int D, int G>
-int fused_stages() {
-  using S = FusedSmem<T, D, G>;
-  int NS = kMaxStages;
-  while (NS > 2 && S::bytes(NS) > kMaxSmem) --NS;
-  return NS;
+constexpr int kMW = 8;                 // compute warps: two groups of four
+constexpr int kMGW = 4;                // warps per tile (16 rows each)
+constexpr int kMCT = kMW * 32;         // compute threads
+constexpr int kMFT = kMCT + 32;        // + the staging warp
+constexpr int kMTT = kMGW * 16;        // rows per tile
+constexpr int kHalfBytes = kMTT * 128; // one 64-column half of a tile (1024-byte multiple)
+
+enum : int { kPieceFlush = 1 };        // meta flag: last piece of this CTA's part of the head
+
+template <int D>
+struct MmaGeo {
+  static constexpr int NH = D / 64;                  // 64-column halves
+  static constexpr int VOFF = NH * kHalfBytes;
+  static constexpr int STAGE = 2 * NH * kHalfBytes;  // K halves, then V halves
+  static constexpr int TX = STAGE;                   // bytes each stage's copies deliver
+};
+
+template <int D, int G>
+struct MmaSmem {
+  using Geo = MmaGeo<D>;
+  static constexpr int up16(int x) { return (x + 15) & ~15; }
+  static constexpr int RED = up16(kMW * G * (D + 2) * 4);       // warp states
+  static constexpr int QF = kMW * (D / 16) * 32 * 8;            // per-warp Q fragments
+  static constexpr int SEL = (kMaxK + 4) * 4 * 2;               // selected prefix + starts
+  static constexpr int MISC = kMiscBytes;
+  static constexpr int ALIGN = 1024;                            // ring base alignment slack
+  static size_t bytes(int NS) {
+    return size_t(NS) * Geo::STAGE + RED + QF + SEL + MISC + ALIGN;
+  }
+};
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+#pragma nv_diag_suppress 550  // the discarded accumulators of mma_rows8
+// d[0..1] += A . B for the rows lane/4 of a 16x8 tile; A rows 8..15 are zero
+// (a1 = a3 = 0) and their accumulators are not kept.
+__device__ __forceinline__ void mma_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0,
+                                          uint32_t b1) {
+  float d2, d3;  // rows 8..15: discarded
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%5}, "
+      "{%7,%8}, {%0,%1,%9,%9};"
+      : "+f"(d[0]), "+f"(d[1]), "=f"(d2), "=f"(d3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(b0), "r"(b1), "f"(0.f));
+}
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+// byte offset of 16-byte chunk ch of row r in a 128-byte-swizzled half tile
+__device__ __forceinline__ uint32_t swz(int r, int ch) {
+  return uint32_t(r * 128 + ((ch ^ (r & 7)) << 4));
 }
 
+// One warp's softmax state: head hq = lane/4 (q heads >= G are padding).
+// The warp's Q fragments live in its own shared-memory copy `qf`
+// ([KS][32 lanes] x (a0, a2)), read back for every tile.
+template <int D>
+struct MmaState {
+  static constexpr int KS = D / 16;  // k-steps of Q.K^T
+  static constexpr int NTD = D / 8;  // n-tiles of P.V
+  const uint2* qf;                   // this warp's Q fragments
+  float m;                           // running max of head hq (log2 units)
+  float l;                           // sum of this lane's weights of head hq
+  float o[NTD][2];                   // O[hq][8 nt + 2 (lane % 4) + {0, 1}]
+};
+
+template <int D, int G>
+__device__ __forceinline__ void mma_load_q(const AttendArgs& at, int bh, MmaState<D>& st,
+                                           uint2* qf) {
+  const int lane = threadIdx.x & 31, hq = lane >> 2, c = (lane & 3) * 2;
+  const int b = bh / at.Hkv, h = bh % at.Hkv;
+  const __nv_bfloat16* qp =
+      static_cast<const __nv_bfloat16*>(at.q) + (int64_t(b) * at.Hq + h * G + hq) * D + c;
+  // (each lane reads back only its own entries)
+#pragma unroll
+  for (int ks = 0; ks < MmaState<D>::KS; ++ks)
+    qf[ks * 32 + lane] =
+        hq < G ? make_uint2(__ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16)),
+                            __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8)))
+               : make_uint2(0u, 0u);
+  st.qf = qf;
+  st.m = -INFINITY;
+  st.l = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < MmaState<D>::NTD; ++nt) st.o[nt][0] = st.o[nt][1] = 0.f;
+}
+
+// keeps the bf16 halves of b whose rows (lo half: row, hi half: row + 1) are valid
+__device__ __forceinline__ uint32_t keep_rows(uint32_t b, int row, int nvalid) {
+  const uint32_t lo = row < nvalid ? 0x0000ffffu : 0u;
+  const uint32_t hi = row + 1 < nvalid ? 0xffff0000u : 0u;
+  return b & (lo | hi);
+}
+
+// Rows [16 wr, 16 wr + 16) of the tile at shared address `stage` (nvalid rows
+// valid; the rest hold whatever the boxes brought and get zero weight).
+template <int D>
+__device__ __forceinline__ void mma_consume(uint32_t stage, int nvalid, MmaState<D>& st, int wr,
+                                            float scale_log2) {
+  using Geo = MmaGeo<D>;
+  constexpr int KS = MmaState<D>::KS, NTD = MmaState<D>::NTD;
+  const int lane = threadIdx.x & 31;
+  const int r0 = wr * 16;
+  if (r0 >= nvalid) return;
+  // S^T: n-tile nt holds rows r0 + 8 nt + [0, 8).  K-steps ks, ks + 1 cover
+  // columns [16 ks, 16 ks + 32): half ks / 4, chunks 2 (ks % 4) + [0, 4).
+  float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+  for (int ks = 0; ks < KS; ks += 2) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      uint32_t bk[4];  // b0, b1 of k-steps ks and ks + 1
+      const int r = r0 + 8 * nt + (lane & 7);
+      ldsm_x4(bk, stage + (ks / 4) * kHalfBytes + swz(r, 2 * (ks % 4) + (lane >> 3)));
+      const uint2 qa = st.qf[ks * 32 + lane], qb = st.qf[(ks + 1) * 32 + lane];
+      mma_rows8(sc[nt], qa.x, qa.y, bk[0], bk[1]);
+      mma_rows8(sc[nt], qb.x, qb.y, bk[2], bk[3]);
+    }
+  }
+  // this lane's rows: r0 + c + {0, 1} (n-tile 0) and r0 + 8 + c + {0, 1} (n-tile 1)
+  const int c = (lane & 3) * 2;
+  float x[4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int row = r0 + 8 * nt + c + e;
+      x[nt * 2 + e] = row < nvalid ? sc[nt][e] * scale_log2 : -INFINITY;
+    }
+  float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+  mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+  mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+  if (mt > st.m) {  // per head (lanes differ); no collective inside
+    const float cf = ex2_fast(st.m - mt);  // 0 while the state is empty
+    st.l *= cf;
+#pragma unroll
+    for (int nt = 0; nt < NTD; ++nt) {
+      st.o[nt][0] *= cf;
+      st.o[nt][1] *= cf;
+    }
+    st.m = mt;
+  }
+  const float mu = st.m == -INFINITY ? 0.f : st.m;
+  float p[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) p[e] = ex2_fast(x[e] - mu);
+  st.l += (p[0] + p[1]) + (p[2] + p[3]);
+  // A fragments of P^T: a0 = rows c, c+1 (n-tile 0), a2 = rows 8+c, 9+c (n-tile 1)
+  const uint32_t h0 = pack_bf16(p[0], p[1]), h2 = pack_bf16(p[2], p[3]);
+  const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h0));
+  const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h2));
+  const uint32_t l0 = pack_bf16(p[0] - f0.x, p[1] - f0.y);
+  const uint32_t l2 = pack_bf16(p[2] - f2.x, p[3] - f2.y);
+  // V (transposed): n-tiles nt, nt + 1 cover columns [8 nt, 8 nt + 16): half
+  // nt / 8, chunks nt % 8 + {0, 1}.  Rows past nvalid may hold non-finite
+  // values from the boxes: a partial slice masks them out of its fragments.
+  const bool partial = r0 + 16 > nvalid;
+  const int vr = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+  for (int nt = 0; nt < NTD; nt += 2) {
+    uint32_t bv[4];  // b0, b1 of n-tiles nt and nt + 1
+    ldsm_x4_t(bv, stage + Geo::VOFF + (nt / 8) * kHalfBytes + swz(vr, (nt % 8) + (lane >> 4)));
+    if (partial) {
+      bv[0] = keep_rows(bv[0], r0 + c, nvalid);
+      bv[1] = keep_rows(bv[1], r0 + 8 + c, nvalid);
+      bv[2] = keep_rows(bv[2], r0 + c, nvalid);
+      bv[3] = keep_rows(bv[3], r0 + 8 + c, nvalid);
+    }
+    mma_rows8(st.o[nt], h0, h2, bv[0], bv[1]);
+    mma_rows8(st.o[nt], l0, l2, bv[0], bv[1]);
+    mma_rows8(st.o[nt + 1], h0, h2, bv[2], bv[3]);
+    mma_rows8(st.o[nt + 1], l0, l2, bv[2], bv[3]);
+  }
+}
+
+// Warp 0 of the whole-block kernel: cuts this CTA's rows into pieces (one
+// segment, <= 64 rows) and stages each into the ring with bulk tensor copies.
+// The last piece of each unit (head part) carries the flush flag; a unit
+// without rows still gets one empty piece.
+template <int D>
+__device__ __forceinline__ void produce_pieces(const FusedArgs& a, const CUtensorMap* kmap,
+                                               const CUtensorMap* vmap, char* stages,
+                                               const MiscLayout& ms, int* sel_pref,
+                                               int* sel_phys) {
+  using Geo = MmaGeo<D>;
+  const int lane = threadIdx.x & 31;
+  const int NS = a.NS;
+  int j = 0, s = 0, sel_bh = -1;
+  uint32_t ph = 0;
+  bool selection_visible = false;
+  // stages one piece of n rows starting at pool row y (n = 0: no copies)
+  auto emit = [&](int n, int y, int bh, int part, bool flush) -> bool {
+    // stage s is free once all compute warps released its previous piece
+    if (j >= NS && !mbar_wait(&ms.empty[s], ph ^ 1u, ms.abort_flag, a.at.status, 1))
+      return false;
+    if (lane == 0) {
+      Meta& mt = ms.meta[s];
+      mt.nrows = n;
+      mt.pad[0] = bh;
+      mt.pad[1] = part;
+      mt.pad[2] = flush ? kPieceFlush : 0;
+      mbar_arrive_tx(&ms.full[s], n > 0 ? uint32_t(Geo::TX) : 0u);
+      if (n > 0) {
+        char* stg = stages + size_t(s) * Geo::STAGE;
+#pragma unroll
+        for (int hh = 0; hh < Geo::NH; ++hh) {
+          tma_load_2d(stg + hh * kHalfBytes, kmap, hh * 64, y, &ms.full[s]);
+          tma_load_2d(stg + Geo::VOFF + hh * kHalfBytes, vmap, hh * 64, y, &ms.full[s]);
+        }
+      }
+    }
+    __syncwarp();
+    ++j;
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1u;
+    }
+    return true;
+  };
+  Iter it;
+  iter_begin(a, it);
+  bool alive = true;
+  while (!it.done && alive) {
+    const int bh = it.bh, part = it.part;
+    const int s0 = a.ps[part], s1 = a.ps[part + 1];
+    const int sel0 = a.px[part] - s0, sel1 = a.px[part + 1] - s1;
+    bool pend = false;
+    int pn = 0, py = 0;
+    for (int kind = 1; kind <= 2 && alive; ++kind) {
+      int v = kind == 1 ? s0 : sel0;
+      const int vend = kind == 1 ? s1 : sel1;
+      if (v >= vend) continue;
+      int st_pref[3], st_phys[2];
+      const int* pref;
+      const int* phys;
+      int nseg;
+      if (kind == 1) {
+        st_pref[0] = 0;
+        st_pref[1] = a.at.sink_end;
+        st_pref[2] = a.L_st;
+        st_phys[0] = 0;
+        st_phys[1] = static_cast<int>(a.at.w0);
+        pref = st_pref;
+        phys = st_phys;
+        nseg = 2;
+      } else {
+        if (!selection_visible) {
+          // the selection comes from the kernel this one depends on: wait for
+          // its completion (and its writes) before the first selected row
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          selection_visible = true;
+        }
+        if (bh != sel_bh) {
+          // prefix of the clipped lengths of this head's selected blocks, and
+          // their first tokens
+          const int k = a.at.k;
+          int run = 0;
+          for (int base = 0; base < k; base += 32) {
+            const int jj = base + lane;
+            int len = 0, start = 0;
+            if (jj < k) {
+              const int blk = __ldcg(a.idx + int64_t(bh) * k + jj);
+              const bool okb = blk >= a.at.first && blk < a.at.first + a.at.nc;
+              const int64_t lo = max(int64_t(blk) * a.at.bs, int64_t(a.at.sink));
+              const int64_t hi = min(int64_t(blk + 1) * a.at.bs, a.at.w0);
+              start = static_cast<int>(lo);
+              len = okb && hi > lo ? static_cast<int>(hi - lo) : 0;
+              if (!okb) report(a.at.status, RBA_ERR_BOUNDS, kWhereFused, blk);
+            }
+            int incl = len;
+            for (int o = 1; o < 32; o <<= 1) {
+              const int t = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += t;
+            }
+            if (jj < k) {
+              sel_pref[jj] = run + incl - len;
+              sel_phys[jj] = start;
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
+          }
+          if (lane == 0) sel_pref[k] = run;
+          __syncwarp();
+          sel_bh = bh;
+        }
+        pref = sel_pref;
+        phys = sel_phys;
+        nseg = a.at.k;
+      }
+      const int vlim = min(vend, pref[nseg]);
+      while (v < vlim) {
+        // the segment holding v: the last one starting at or before it
+        int lo2 = 0, hi2 = nseg - 1;
+        while (lo2 < hi2) {
+          const int mid = (lo2 + hi2 + 1) >> 1;
+          if (pref[mid] <= v) lo2 = mid; else hi2 = mid - 1;
+        }
+        const int n = min(min(vlim, pref[lo2 + 1]), v + kMTT) - v;
+        const int y = static_cast<int>(int64_t(bh) * a.at.cap + phys[lo2] + (v - pref[lo2]));
+        if (pend && !emit(pn, py, bh, part, false)) {
+          alive = false;
+          break;
+        }
+        pend = true;
+        pn = n;
+        py = y;
+        v += n;
+      }
+    }
+    if (alive && !emit(pend ? pn : 0, py, bh, part, true)) alive = false;
+    if (++it.u >= it.u1) it.done = true; else unit_begin(a, it);
+  }
+  // no copy may still be landing in shared memory when the CTA exits
+  if (lane == 0)
+    for (int q = max(0, j - NS); q < j; ++q) mbar_drain(&ms.full[q % NS], (q / NS) & 1u);
+  __syncwarp();
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kMFT, 1)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap vmap, FusedArgs a) {
+  static_assert(G <= 8, "q heads of a kv head fit the rows 0..7 of the A tile");
+  using Geo = MmaGeo<D>;
+  using S = MmaSmem<D, G>;
+  extern __shared__ char smem_raw[];
+  char* stages = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~uintptr_t(1023));
+  const int NS = a.NS;
+  float* red = reinterpret_cast<float*>(stages + size_t(NS) * Geo::STAGE);
+  uint2* qfrag = reinterpret_cast<uint2*>(reinterpret_cast<char*>(red) + S::RED);
+  int* sel_pref = reinterpret_cast<int*>(reinterpret_cast<char*>(qfrag) + S::QF);
+  int* sel_phys = sel_pref + (kMaxK + 1);
+  const MiscLayout ms(reinterpret_cast<char*>(sel_pref) + S::SEL);
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&ms.full[s], 1);
+      mbar_init(&ms.empty[s], kMW);
+    }
+    mbar_init(ms.merge_bar, 1);
+    *ms.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+  if (warp == 0) {
+    produce_pieces<D>(a, &kmap, &vmap, stages, ms, sel_pref, sel_phys);
+    return;
+  }
+  // ---- compute warps: every warp reads every piece's meta; group grp
+  // computes the pieces i with i % 2 == grp, warp wr of the group rows
+  // [16 wr, 16 wr + 16) of each.  All warps release every stage.
+  const int cw = warp - 1;
+  const int grp = cw / kMGW, wr = cw % kMGW;
+  Iter it;
+  iter_begin(a, it);
+  const int n_units = it.done ? 0 : it.u1 - it.u;
+  const uint32_t ring = smem_u32(stages);
+  MmaState<D> st;
+  int cur_bh = -1, i = 0, s = 0, units = 0;
+  uint32_t ph = 0, merge_ph = 0;
+  bool ok = true;
+  while (units < n_units) {
+    int flags = kPieceFlush, bh = -1, part = 0, nrows = 0;
+    if (ok) ok = mbar_wait(&ms.full[s], ph, ms.abort_flag, a.at.status, 3);
+    if (ok) {
+      const Meta& mt = ms.meta[s];
+      nrows = mt.nrows;
+      bh = mt.pad[0];
+      part = mt.pad[1];
+      flags = mt.pad[2];
+      if (bh != cur_bh) {
+        cur_bh = bh;
+        mma_load_q<D, G>(a.at, bh, st, qfrag + cw * (MmaState<D>::KS * 32));
+      }
+      if ((i & 1) == grp)
+        mma_consume<D>(ring + uint32_t(s) * Geo::STAGE, nrows, st, wr, a.at.scale_log2);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.empty[s]);
+    }
+    ++i;
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1u;
+    }
+    if (flags & kPieceFlush) {
+      // ---- this warp's state of the head -> red[cw][hq]; after a failed
+      // wait every warp still takes part in one flush per unit (with its
+      // state as it stands) so that the barriers inside match
+      if (cur_bh < 0) {
+        cur_bh = 0;
+        mma_load_q<D, G>(a.at, 0, st, qfrag + cw * (MmaState<D>::KS * 32));
+      }
+      float lt = st.l;
+      lt += __shfl_xor_sync(0xffffffffu, lt, 1);
+      lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+      const int hq = lane >> 2, c = (lane & 3) * 2;
+      if (hq < G) {
+        float* r = red + (cw * G + hq) * (D + 2);
+        if (c == 0) {
+          r[0] = st.m;
+          r[1] = lt;
+        }
+#pragma unroll
+        for (int nt = 0; nt < MmaState<D>::NTD; ++nt) {
+          r[2 + nt * 8 + c] = st.o[nt][0];
+          r[2 + nt * 8 + c + 1] = st.o[nt][1];
+        }
+      }
+      // the unit's head and part: from the meta, or from the work list when the wait failed
+      int fbh = bh, fpart = part;
+      if (!ok) {
+        Iter iu;
+        iter_begin(a, iu);
+        iu.u += units;
+        if (iu.u < iu.u1) unit_begin(a, iu);
+        fbh = iu.bh;
+        fpart = iu.part;
+      }
+      finish_head<G, D, kMW, kMCT>(a, fbh, fpart, red, ms, stages, size_t(NS) * Geo::STAGE,
+                                   merge_ph);
+      cur_bh = -1;
+      ++units;
+    }
+  }
+}
+
+constexpr size_t kMaxSmem = 227 * 1024;  // dynamic shared memory of one CTA
+
+// Kernel, threads and shared memory of one (T, D, G) and path: the
+// whole-block tensor-core kernel (MMA) or the CUDA-core one.
+template <typename T, int D, int G, bool MMA>
+struct FusedKernel {
+  static constexpr int kThreads = MMA ? kMFT : kFT;
+  static size_t smem(int NS) {
+    if constexpr (MMA) return MmaSmem<D, G>::bytes(NS);
+    else return FusedSmem<T, D, G>::bytes(NS);
+  }
+  static const void* fn() {
+    if constexpr (MMA) return reinterpret_cast<const void*>(decode_mma_kernel<D, G>);
+    else return reinterpret_cast<const void*>(decode_fused_kernel<T, D, G>);
+  }
+  static int stages() {
+    int NS = kMaxStages;
+    while (NS > 2 && smem(NS) > kMaxSmem) --NS;
+    return NS;
+  }
+};
+
 // CTAs of this kernel that fit on one SM (0: none; <0: a CUDA error)
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool MMA>
 int fused_occupancy_t() {
-  using S = FusedSmem<T, D, G>;
-  const size_t smem = S::bytes(fused_stages<T, D, G>());
+  using K = FusedKernel<T, D, G, MMA>;
+  const size_t smem = K::smem(K::stages());
   if (smem > kMaxSmem) return 0;  // (large fp32 tiles) the split-K kernel runs instead
-  auto kfn = decode_fused_kernel<T, D, G>;
-  if (ensure_smem(reinterpret_cast<const void*>(kfn), smem) != cudaSuccess) return -1;
+  if (ensure_smem(K::fn(), smem) != cudaSuccess) return -1;
   int occ = 0;
-  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kfn, kFT, smem);
+  const cudaError_t e =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, K::fn(), K::kThreads, smem);
   if (getenv("RBA_DEBUG") != nullptr) {
     cudaFuncAttributes fa = {};
-    cudaFuncGetAttributes(&fa, kfn);
+    cudaFuncGetAttributes(&fa, K::fn());
     fprintf(stderr,
-            "rba: decode_fused_kernel regs=%d maxThreads=%d static_smem=%zu local=%zu "
+            "rba: decode attention kernel (%s) regs=%d maxThreads=%d static_smem=%zu local=%zu "
             "max_dyn_smem=%d requested_smem=%zu threads=%d occupancy=%d (%s)\n",
-            fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.localSizeBytes,
-            fa.maxDynamicSharedSizeBytes, smem, kFT, occ, cudaGetErrorString(e));
+            MMA ? "tensor-core, whole blocks" : "cuda-core", fa.numRegs, fa.maxThreadsPerBlock,
+            fa.sharedSizeBytes, fa.localSizeBytes, fa.maxDynamicSharedSizeBytes, smem,
+            K::kThreads, occ, cudaGetErrorString(e));
   }
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
@@ -692,19 +1244,19 @@ int fused_occupancy_t() {
   return occ;
 }
 
-template <typename T, int D, int G>
-rba_status launch_fused_t(FusedArgs a, int P, bool pdl, cudaStream_t stream) {
-  using S = FusedSmem<T, D, G>;
-  const int NS = fused_stages<T, D, G>();
+template <typename T, int D, int G, bool MMA>
+rba_status launch_fused_t(FusedArgs a, const CUtensorMap* maps, int P, bool pdl,
+                          cudaStream_t stream) {
+  using K = FusedKernel<T, D, G, MMA>;
+  const int NS = K::stages();
   a.NS = NS;
-  const size_t smem = S::bytes(NS);
-  auto kfn = decode_fused_kernel<T, D, G>;
-  const int occ = fused_occupancy_t<T, D, G>();
+  const size_t smem = K::smem(NS);
+  const int occ = fused_occupancy_t<T, D, G, MMA>();
   if (occ < 0) return RBA_ERR_CUDA;
   if (occ < 1) return RBA_ERR_UNSUPPORTED;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(P);
-  cfg.blockDim = dim3(kFT);
+  cfg.blockDim = dim3(K::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -712,8 +1264,24 @@ rba_status launch_fused_t(FusedArgs a, int P, bool pdl, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  RBA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kfn, a));
+  if constexpr (MMA) {
+    CUtensorMap km = maps[0], vm = maps[1];
+    void* args[] = {&km, &vm, &a};
+    RBA_CUDA_TRY(cudaLaunchKernelExC(&cfg, K::fn(), args));
+  } else {
+    void* args[] = {&a};
+    RBA_CUDA_TRY(cudaLaunchKernelExC(&cfg, K::fn(), args));
+  }
   return RBA_OK;
+}
+
+// The whole-block tensor-core kernel covers bf16 stores whose blocks are whole
+// 64-row tiles (and whose pools fit 32-bit tensor coordinates).
+bool use_mma(const rba_store* st) {
+  const rba_store_desc& d = st->d;
+  return d.dtype == RBA_BF16 && (d.head_dim == 64 || d.head_dim == 128) &&
+         d.block_size % kMTT == 0 &&
+         int64_t(d.batch) * d.n_kv_heads * d.capacity_tokens < (int64_t(1) << 31) - kMTT;
 }
 
 }  // namespace
@@ -788,22 +1356,29 @@ bool fused_eligible(const rba_store* st, const Geometry& g, int k) {
   return ms <= kMaxGrid;
 }
 
+bool fused_whole_blocks(const rba_store* st) { return use_mma(st); }
+
 int fused_occupancy(const rba_store* st) {
   const rba_store_desc& d = st->d;
   const int G = d.n_q_heads / d.n_kv_heads;
-#define RBA_OCC(T_, D_)                                   \
-  switch (G) {                                            \
-    case 1: return fused_occupancy_t<T_, D_, 1>();        \
-    case 2: return fused_occupancy_t<T_, D_, 2>();        \
-    case 4: return fused_occupancy_t<T_, D_, 4>();        \
-  }                                                       \
+  const bool mma = use_mma(st);
+#define RBA_OCC(T_, D_, M_)                                 \
+  switch (G) {                                              \
+    case 1: return fused_occupancy_t<T_, D_, 1, M_>();      \
+    case 2: return fused_occupancy_t<T_, D_, 2, M_>();      \
+    case 4: return fused_occupancy_t<T_, D_, 4, M_>();      \
+  }                                                         \
   return 0;
   if (d.dtype == RBA_BF16) {
-    if (d.head_dim == 128) { RBA_OCC(__nv_bfloat16, 128) }
-    RBA_OCC(__nv_bfloat16, 64)
+    if (mma) {
+      if (d.head_dim == 128) { RBA_OCC(__nv_bfloat16, 128, true) }
+      RBA_OCC(__nv_bfloat16, 64, true)
+    }
+    if (d.head_dim == 128) { RBA_OCC(__nv_bfloat16, 128, false) }
+    RBA_OCC(__nv_bfloat16, 64, false)
   }
-  if (d.head_dim == 128) { RBA_OCC(float, 128) }
-  RBA_OCC(float, 64)
+  if (d.head_dim == 128) { RBA_OCC(float, 128, false) }
+  RBA_OCC(float, 64, false)
 #undef RBA_OCC
 }
 
@@ -842,27 +1417,47 @@ rba_status launch_fused(const rba_store* st, const void* q, int k, const Geometr
   a.L_st = static_cast<int>(g.sink_end + (g.T - g.w0));
   a.U_sel = k > 0 ? k * d.block_size : 0;
   fused_slot_bytes(st, g, k, &a.m);
-  // part boundaries (host side: no 64-bit divisions on the device)
+  // part boundaries (host side: no 64-bit divisions on the device).  For the
+  // whole-block kernel both kinds of rows are cut at multiples of its tile,
+  // so that interior tiles stay whole.
+  const bool mma = use_mma(st);
   const int64_t Lh = int64_t(a.L_st) + a.U_sel;
   for (int c = 0; c <= a.m; ++c) {
     const int64_t x = Lh * c / a.m;
-    a.px[c] = static_cast<int>(x);
-    a.ps[c] = static_cast<int>(x * a.L_st / Lh);
+    int64_t xs = x * a.L_st / Lh;  // sink/window rows before the boundary
+    int64_t xq = x - xs;           // selected rows before it
+    if (mma && c < a.m) {
+      xs = xs / kMTT * kMTT;
+      xq = xq / kMTT * kMTT;
+    }
+    a.px[c] = static_cast<int>(xs + xq);
+    a.ps[c] = static_cast<int>(xs);
+  }
+  CUtensorMap maps[2];
+  if (mma) {
+    const int64_t rows = int64_t(d.batch) * d.n_kv_heads * d.capacity_tokens;
+    if (!make_tmap_bf16(&maps[0], st->k, rows, d.head_dim, kMTT) ||
+        !make_tmap_bf16(&maps[1], st->v, rows, d.head_dim, kMTT))
+      return RBA_ERR_CUDA;
   }
   const int G = d.n_q_heads / d.n_kv_heads;
-#define RBA_FUSED(T_, D_)                                               \
-  switch (G) {                                                          \
-    case 1: return launch_fused_t<T_, D_, 1>(a, P, pdl, stream);        \
-    case 2: return launch_fused_t<T_, D_, 2>(a, P, pdl, stream);        \
-    case 4: return launch_fused_t<T_, D_, 4>(a, P, pdl, stream);        \
-  }                                                                     \
+#define RBA_FUSED(T_, D_, M_)                                                   \
+  switch (G) {                                                                  \
+    case 1: return launch_fused_t<T_, D_, 1, M_>(a, maps, P, pdl, stream);      \
+    case 2: return launch_fused_t<T_, D_, 2, M_>(a, maps, P, pdl, stream);      \
+    case 4: return launch_fused_t<T_, D_, 4, M_>(a, maps, P, pdl, stream);      \
+  }                                                                             \
   return RBA_ERR_UNSUPPORTED;
   if (d.dtype == RBA_BF16) {
-    if (d.head_dim == 128) { RBA_FUSED(__nv_bfloat16, 128) }
-    RBA_FUSED(__nv_bfloat16, 64)
+    if (mma) {
+      if (d.head_dim == 128) { RBA_FUSED(__nv_bfloat16, 128, true) }
+      RBA_FUSED(__nv_bfloat16, 64, true)
+    }
+    if (d.head_dim == 128) { RBA_FUSED(__nv_bfloat16, 128, false) }
+    RBA_FUSED(__nv_bfloat16, 64, false)
   }
-  if (d.head_dim == 128) { RBA_FUSED(float, 128) }
-  RBA_FUSED(float, 64)
+  if (d.head_dim == 128) { RBA_FUSED(float, 128, false) }
+  RBA_FUSED(float, 64, false)
 #undef RBA_FUSED
 }
 

@@ -14,6 +14,8 @@ size_t fused_sync_bytes(const rba_store* st);
 size_t fused_slot_bytes(const rba_store* st, const Geometry& g, int k, int* ms);
 // CTAs of the attention kernel per SM for this store's types (0: none, <0: CUDA error)
 int fused_occupancy(const rba_store* st);
+// whether the persistent kernel of this store is the whole-block tensor-core one
+bool fused_whole_blocks(const rba_store* st);
 // pdl: launched as a programmatic dependent of the top-k kernel (its stager
 // waits for that kernel before reading idx)
 rba_status launch_fused(const rba_store* st, const void* q, int k, const Geometry& g, float scale,

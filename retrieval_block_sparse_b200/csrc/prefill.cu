@@ -27,7 +27,6 @@
 // RBA_ERR_TIMEOUT, stops issuing work, drains, frees TMEM and returns.
 #include <cuda.h>
 #include <cstring>
-#include <mutex>
 
 #include "rba_internal.cuh"
 
@@ -681,38 +680,9 @@ __global__ void gather_kernel(PrefillArgs a, const __nv_bfloat16* __restrict__ K
   }
 }
 
-// driver entry point for tensor-map encoding (no link-time libcuda)
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(p);
-  });
-  return fn;
-}
-
 // [rows][128] bf16 matrix, 128-byte-swizzled boxes of 64 columns x 128 rows
 bool make_map(CUtensorMap* m, const void* base, int64_t rows) {
-  EncodeFn fn = encode_fn();
-  if (fn == nullptr || base == nullptr || rows <= 0) return false;
-  const cuuint64_t dims[2] = {cuuint64_t(kHD), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(kHD) * 2};
-  const cuuint32_t box[2] = {64, 128};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  return make_tmap_bf16(m, base, rows, kHD, 128);
 }
 
 struct Plan {

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <cuda.h>
+
 #include "rba.h"
 
 struct rba_store {
@@ -144,6 +146,12 @@ cudaError_t ensure_smem(const void* kernel, size_t bytes);
   } while (0)
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Tensor map of a row-major [rows][cols] bf16 matrix for 2-D bulk tensor
+// copies: boxes of 64 columns (128 bytes) x box_rows rows, 128-byte swizzle,
+// zero fill outside the matrix.  False if the driver's encoder is unavailable
+// or rejects the arguments.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows);
 inline size_t dtype_size(rba_dtype t) { return t == RBA_BF16 ? 2 : 4; }
 
 }  // namespace rba

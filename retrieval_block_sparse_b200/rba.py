@@ -264,8 +264,9 @@ class Store:
         return torch.zeros(max(n, 16), dtype=torch.uint8, device=self.k.device)
 
     def decode_plan(self, k, T, sink, window):
-        """1: score -> top-k -> persistent attention, overlapped (programmatic dependent
-        launches); 0: score -> top-k -> split-K in stream order; <0: see rba.h."""
+        """2: score -> top-k -> whole-block tensor-core attention kernel, overlapped
+        (programmatic dependent launches); 1: the same with the CUDA-core attention
+        kernel; 0: score -> top-k -> split-K in stream order; <0: see rba.h."""
         return lib().rba_decode_step_plan(self.handle, k, T, sink, window)
 
     def decode_step(self, q, k, T, sink, window, *, scale=None, workspace=None, out=None,
