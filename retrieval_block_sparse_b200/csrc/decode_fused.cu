@@ -1102,21 +1102,29 @@ __global__ void __launch_bounds__(kMFT, 1)
   const MiscLayout ms(reinterpret_cast<char*>(sel_pref) + S::SEL);
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&ms.full[s], 1);
-      mbar_init(&ms.empty[s], kMW);
-    }
-    mbar_init(ms.merge_bar, 1);
-    *ms.abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-  __syncthreads();
   if (warp == 0) {
+    // the staging warp sets up the barriers, releases the compute warps
+    // (named barrier 2, which it does not wait on) and starts copying
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap))
+                   : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap))
+                   : "memory");
+      for (int s = 0; s < NS; ++s) {
+        mbar_init(&ms.full[s], 1);
+        mbar_init(&ms.empty[s], kMW);
+      }
+      mbar_init(ms.merge_bar, 1);
+      *ms.abort_flag = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncwarp();
+    asm volatile("bar.arrive 2, %0;" ::"n"(kMFT) : "memory");
     produce_pieces<D>(a, &kmap, &vmap, stages, ms, sel_pref, sel_phys);
     return;
   }
+  asm volatile("bar.sync 2, %0;" ::"n"(kMFT) : "memory");
   // ---- compute warps: every warp reads every piece's meta; group grp
   // computes the pieces i with i % 2 == grp, warp wr of the group rows
   // [16 wr, 16 wr + 16) of each.  All warps release every stage.

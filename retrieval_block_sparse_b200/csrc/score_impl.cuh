@@ -33,6 +33,28 @@ __global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int can
   __shared__ float qs[D];
   const int bh = blockIdx.y;
   const int b = bh / a.Hkv, h = bh - b * a.Hkv, g = a.Hq / a.Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % LPC, slot = lane / LPC;
+  const uint4* base = reinterpret_cast<const uint4*>(
+      static_cast<const RT*>(a.rep) + (int64_t(bh) * a.rep_rows + a.first) * (R * D));
+  const int c_begin = blockIdx.x * cand_per_cta;
+  const int c_end = min(a.nc, c_begin + cand_per_cta);
+  float* out = a.scores + int64_t(bh) * a.nc;
+  // U candidate groups of this warp's first iteration: their loads are issued
+  // before the query is summed, so the two latencies overlap
+  uint4 v[U][VPL];
+  auto load_groups = [&](int c0) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * CPW + slot;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        v[u][i] = c < c_end ? ld_stream(base + int64_t(c) * VPC + sub + i * LPC)
+                            : make_uint4(0, 0, 0, 0);
+    }
+  };
+  const int c_first = c_begin + warp * CPW * U;
+  load_groups(c_first);
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float acc = 0.f;
     if (a.qsum != nullptr) {
@@ -46,8 +68,6 @@ __global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int can
     qs[d] = acc;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane % LPC, slot = lane / LPC;
   float qr[VPL][EPV];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
@@ -55,21 +75,8 @@ __global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int can
 #pragma unroll
     for (int e = 0; e < EPV; ++e) qr[i][e] = qs[d0 + e];
   }
-  const uint4* base = reinterpret_cast<const uint4*>(
-      static_cast<const RT*>(a.rep) + (int64_t(bh) * a.rep_rows + a.first) * (R * D));
-  const int c_begin = blockIdx.x * cand_per_cta;
-  const int c_end = min(a.nc, c_begin + cand_per_cta);
-  float* out = a.scores + int64_t(bh) * a.nc;
-  for (int c0 = c_begin + warp * CPW * U; c0 < c_end; c0 += NW * CPW * U) {
-    uint4 v[U][VPL];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = c0 + u * CPW + slot;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        v[u][i] = c < c_end ? ld_stream(base + int64_t(c) * VPC + sub + i * LPC)
-                            : make_uint4(0, 0, 0, 0);
-    }
+  for (int c0 = c_first; c0 < c_end; c0 += NW * CPW * U) {
+    if (c0 != c_first) load_groups(c0);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       float acc = 0.f;
