@@ -340,7 +340,8 @@ def run_ours(args):
         g_one.append(g)
     plan = master.decode_plan(w.top_k, w.context, w.sink, w.window)
     # score + top-k (one kernel for rows <= 8192 candidates, four above) + attention
-    kern_per_step = (1 if w.top_k == 0 else (3 if nc <= 8192 else 6))
+    # as the library reports
+    kern_per_step = master.decode_launches(w.top_k, w.context, w.sink, w.window)
     n_nodes = count_kernel_nodes(g_one[0])
 
     def run_steps(n):
@@ -476,7 +477,7 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank != 0:
         return None
-    launches = kern_per_step if kern_per_step else (3 if nc <= 8192 else 6)
+    launches = kern_per_step
     line = {
         "metric": METRIC, "value": round(steps_per_s, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_us / 1e3, 6),

@@ -260,6 +260,13 @@ size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t
 int32_t rba_decode_step_plan(const rba_store* store, int32_t k, int64_t T, int32_t sink,
                              int32_t window);
 
+/* Number of kernels rba_decode_step enqueues for this problem (host only, launches
+ * nothing): block scores and top-k (one kernel for rows of up to 8192 candidates, four
+ * above; neither when k = 0), then one attention kernel (persistent or split-K).  -4 for
+ * invalid arguments. */
+int32_t rba_decode_step_launches(const rba_store* store, int32_t k, int64_t T, int32_t sink,
+                                 int32_t window);
+
 /* One step of streaming decode ([IL] overall framework: the newest tokens form
  * the local window and the tokens before it stay in memory as units that are
  * represented once; [ML] 2.3.2: a completed chunk is memorised).  The store

@@ -345,6 +345,17 @@ int32_t rba_decode_step_plan(const rba_store* st, int32_t k, int64_t T, int32_t 
   return fused_whole_blocks(st) ? 2 : 1;
 }
 
+int32_t rba_decode_step_launches(const rba_store* st, int32_t k, int64_t T, int32_t sink,
+                                 int32_t window) {
+  using namespace rba;
+  Geometry g;
+  if (st == nullptr || k < 0 || geometry(st, T, sink, window, &g) != RBA_OK || k > g.nc)
+    return -4;
+  int32_t n = 0;
+  if (k > 0) n += 1 + (g.nc <= kSmallN ? 1 : 4);  // scores; top-k (one kernel, or four)
+  return n + 1;  // the attention kernel (persistent or split-K)
+}
+
 size_t rba_decode_step_workspace_size(const rba_store* st, int32_t k, int64_t T, int32_t sink,
                                       int32_t window) {
   using namespace rba;

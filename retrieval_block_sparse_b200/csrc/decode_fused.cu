@@ -298,7 +298,7 @@ struct FusedSmem {
 // which arrive by bulk copies into the (idle) stage ring.  Called by all NCT
 // compute threads; ends with them synchronised.
 template <int G, int D, int NW, int NCT>
-__device__ __forceinline__ void finish_head(const FusedArgs& a, int bh, int ord, const float* red,
+__device__ __forceinline__ void finish_head(const FusedArgs& a, int bh, int ord, float* red,
                             const MiscLayout& ms, char* stages, size_t ring_bytes,
                             uint32_t& merge_ph) {
   constexpr int kSlotFloats = slot_floats(G, D);
@@ -360,20 +360,23 @@ __device__ __forceinline__ void finish_head(const FusedArgs& a, int bh, int ord,
     if (ms.s_misc[9]) {
       // the last part of the head merges the m slots.  The slots go to shared
       // memory by bulk copies into the stage ring (idle: with m > 1 a CTA
-      // holds one part of one head, all of it consumed), a chunk at a time;
-      // each thread then folds every slot's (m, l, o[d]) of its output
-      // elements (g, d) into a running (max, sum, output).
+      // holds one part of one head, all of it consumed), a chunk at a time.
+      // Per chunk, warp g < G folds the slots' (m, l) of q head g into a
+      // running max and denominator and leaves one factor per slot in `fac`
+      // (red is free by now); then each thread folds its output elements
+      // (g, d) with those factors.
       constexpr int SLOT = kSlotFloats * 4;  // a multiple of 16 bytes
       constexpr int NX = (G * D + NCT - 1) / NCT;
       const int nl = a.m;
-      const int chunk = static_cast<int>(ring_bytes / SLOT);
-      float M[NX], L[NX], O[NX];
+      const int chunk = min(static_cast<int>(ring_bytes / SLOT), (NW * (D + 2)) / 2);
+      float* mfac = const_cast<float*>(red);      // [chunk][G] factors
+      float* mrun = ms.s_f;                       // [G] running max (replaces fac / gmax)
+      float* lrun = ms.s_f + 16;                  // [G] running denominator
+      float* rsc = ms.s_f + 32;                   // [G] rescale of the running sums
+      const int lane = tid & 31, cw = tid >> 5;
+      float O[NX];
 #pragma unroll
-      for (int r = 0; r < NX; ++r) {
-        M[r] = -INFINITY;
-        L[r] = 0.f;
-        O[r] = 0.f;
-      }
+      for (int r = 0; r < NX; ++r) O[r] = 0.f;
       for (int j0 = 0; j0 < nl; j0 += chunk) {
         const int n = min(chunk, nl - j0);
         if (tid == 0) {
@@ -388,33 +391,51 @@ __device__ __forceinline__ void finish_head(const FusedArgs& a, int bh, int ord,
         if (!ok && tid == 0) mbar_drain(ms.merge_bar, merge_ph);  // no copy outlives the CTA
         merge_ph ^= 1u;
         const float* sm = reinterpret_cast<const float*>(stages);
+        if (cw < G) {
+          const int g = cw;
+          float cm = -INFINITY;
+          for (int j = lane; j < n; j += 32) cm = fmaxf(cm, sm[j * kSlotFloats + g * (D + 2)]);
+          for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+          const float mo = j0 == 0 ? -INFINITY : mrun[g];  // (warp g alone writes mrun[g])
+          const float lo = j0 == 0 ? 0.f : lrun[g];
+          const float mn = fmaxf(mo, cm);
+          float lsum = 0.f;
+          for (int j = lane; j < n; j += 32) {
+            const float mj = sm[j * kSlotFloats + g * (D + 2)];
+            const float f = mj == -INFINITY ? 0.f : exp2f(mj - mn);
+            mfac[j * G + g] = f;
+            lsum += f * sm[j * kSlotFloats + g * (D + 2) + 1];
+          }
+          for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+          if (lane == 0) {
+            const float sc = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+            rsc[g] = sc;
+            lrun[g] = lo * sc + lsum;
+            mrun[g] = mn;
+          }
+        }
+        compute_sync<NCT>();
 #pragma unroll
         for (int r = 0; r < NX; ++r) {
           const int x = tid + r * NCT;
           if (!ok || x >= G * D) continue;
           const int gg = x / D, d = x % D;
-          for (int j = 0; j < n; ++j) {
-            const float* q = sm + j * kSlotFloats + gg * (D + 2);
-            const float mj = q[0], lj = q[1], oj = q[2 + d];
-            const float mn = fmaxf(M[r], mj);
-            const float sa = M[r] == -INFINITY ? 0.f : exp2f(M[r] - mn);
-            const float sb = mj == -INFINITY ? 0.f : exp2f(mj - mn);
-            L[r] = L[r] * sa + lj * sb;
-            O[r] = O[r] * sa + oj * sb;
-            M[r] = mn;
-          }
+          float acc = O[r] * rsc[gg];
+          for (int j = 0; j < n; ++j) acc += mfac[j * G + gg] * sm[j * kSlotFloats + gg * (D + 2) + 2 + d];
+          O[r] = acc;
         }
-        compute_sync<NCT>();  // the chunk buffer is read before the next copy
+        compute_sync<NCT>();  // the chunk buffer and factors are read before the next copy
       }
 #pragma unroll
       for (int r = 0; r < NX; ++r) {
         const int x = tid + r * NCT;
         if (x >= G * D) continue;
         const int gg = x / D, d = x % D;
-        a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = L[r] > 0.f ? O[r] / L[r] : 0.f;
+        const float L = lrun[gg];
+        a.at.out[(int64_t(b) * a.at.Hq + h * G + gg) * D + d] = L > 0.f ? O[r] / L : 0.f;
         if (d == 0 && a.at.lse != nullptr)
           a.at.lse[int64_t(b) * a.at.Hq + h * G + gg] =
-              L[r] > 0.f ? (M[r] + log2f(L[r])) * 0.6931471805599453f : -INFINITY;
+              L > 0.f ? (mrun[gg] + log2f(L)) * 0.6931471805599453f : -INFINITY;
       }
       if (tid == 0) a.tickets[bh] = 0;  // zero again for the next call
     }
@@ -1300,12 +1321,12 @@ static int64_t attention_rows(const rba_store* st, const Geometry& g, int k) {
 }
 
 // CTAs available to the attention launch: one per SM, leaving the SMs that
-// the top-k kernel (one CTA per row) holds while this kernel starts; fewer
-// for small problems.
+// the top-k kernel holds while this kernel starts; fewer for small problems.
 static int cta_budget(const rba_store* st, const Geometry& g, int k) {
   const int BH = st->d.batch * st->d.n_kv_heads;
   int sms = num_sms();
-  if (k > 0 && g.nc <= kSmallN && BH <= sms / 4) sms -= BH;
+  const int held = k > 0 ? topk_ctas(BH, g.nc) : 0;
+  if (held > 0 && held <= sms / 4) sms -= held;
   int64_t P = (attention_rows(st, g, k) + kMinRowsPerCta - 1) / kMinRowsPerCta;
   if (P > sms) P = sms;
   if (P > kMaxGrid) P = kMaxGrid;

@@ -273,6 +273,8 @@ rba_status launch_topk(const float* scores, int rows, int n, int k, int index_ba
   return launch_topk_large(scores, rows, n, k, index_base, idx, ws, stream);
 }
 
+int topk_ctas(int rows, int n) { return n <= kSmallN ? rows : 0; }
+
 size_t topk_workspace(int rows, int n, int k) {
   return n <= kSmallN ? 0 : topk_large_workspace(rows, n, k);
 }

@@ -18,5 +18,8 @@ rba_status launch_topk_large(const float* scores, int rows, int n, int k, int in
 rba_status launch_topk(const float* scores, int rows, int n, int k, int index_base, int32_t* idx,
                        void* ws, size_t ws_bytes, cudaStream_t stream, bool pdl);
 size_t topk_workspace(int rows, int n, int k);
+// CTAs the selector of `rows` rows of n scores runs while a dependent kernel
+// starts (0: the multi-CTA path)
+int topk_ctas(int rows, int n);
 
 }  // namespace rba

@@ -45,6 +45,7 @@ SIGNATURES = {
                                  _p, _c_size, _p]),
     "rba_decode_step_workspace_size": (_c_size, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
     "rba_decode_step_plan": (_c_i32, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
+    "rba_decode_step_launches": (_c_i32, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
     "rba_stream_step": (_c_i32, [_p, _p, _p, _p, _c_i64, _c_i32, _c_i32, _c_i32, _c_f32, _p,
                                  _c_i32, _p, _p, _p, ctypes.POINTER(_c_i32), _p, _c_size, _p]),
     "rba_memory_rule": (_c_i32, [_c_i64, ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i64),
@@ -268,6 +269,10 @@ class Store:
         (programmatic dependent launches); 1: the same with the CUDA-core attention
         kernel; 0: score -> top-k -> split-K in stream order; <0: see rba.h."""
         return lib().rba_decode_step_plan(self.handle, k, T, sink, window)
+
+    def decode_launches(self, k, T, sink, window):
+        """Kernels one decode_step enqueues (-4: invalid arguments)."""
+        return lib().rba_decode_step_launches(self.handle, k, T, sink, window)
 
     def decode_step(self, q, k, T, sink, window, *, scale=None, workspace=None, out=None,
                     lse=None, idx=None, scores=None):

@@ -34,6 +34,24 @@ def test_topk_large_rows(rba, n, k, ties):
         np.testing.assert_array_equal(got[r], O.top_k(s[r].astype(np.float64), k))
 
 
+@pytest.mark.parametrize("n,k", [(1024, 600), (1024, 1), (700, 69), (33, 32), (991, 32),
+                                 (129, 128)])
+def test_topk_warp_rows_skewed_and_tied(rba, n, k):
+    # rows of at most 1024 scores are selected by one warp: cover a value
+    # range dominated by a few outliers (crowded boundary bin), two-level ties
+    # (radix path), infinities (radix path) and plain normal rows
+    rng = np.random.default_rng(n * 7 + k)
+    rows = [rng.standard_normal(n),
+            np.where(rng.random(n) < 0.02, 1e4, rng.standard_normal(n) * 1e-3),
+            rng.integers(0, 2, n).astype(np.float64),
+            np.where(rng.random(n) < 0.05, np.inf, rng.standard_normal(n)),
+            np.where(rng.random(n) < 0.05, -np.inf, rng.standard_normal(n))]
+    s = np.stack(rows).astype(np.float32)
+    got = _run(rba, s, k, base=11)
+    for r in range(s.shape[0]):
+        np.testing.assert_array_equal(got[r], O.top_k(s[r].astype(np.float64), k) + 11)
+
+
 def test_topk_signed_zero_and_constant_rows(rba):
     s = np.zeros((2, 300), dtype=np.float32)
     s[0, ::2] = -0.0
