@@ -183,15 +183,22 @@ def memorize(K: np.ndarray, mode: str, bs: int, r: int = 1, probe=None,
 # scoring and selection
 
 
-def score_dot(qs: np.ndarray, reps: np.ndarray) -> np.ndarray:
+def score_dot(qs: np.ndarray, reps: np.ndarray, reduce: str = "sum") -> np.ndarray:
     """Block score by dot product, [LM] query-landmark similarity and [IL]
     relevance against representative tokens.
 
     qs [m][D] are the query vectors that share the selection (the q heads of a
-    GQA group); reps [n][r][D].  s_j = sum_q sum_i q . rep_{j,i}.
+    GQA group); reps [n][r][D].  reduce="sum": s_j = sum_q sum_i q . rep_{j,i};
+    reduce="max" (variant): s_j = max_i sum_q q . rep_{j,i}, a block as relevant
+    as its most relevant representative key.
     """
     pair = reps @ qs.T                    # [n][r][m]: one dot product per (key, query)
-    return pair.reshape(pair.shape[0], -1).sum(axis=1)
+    per_key = pair.sum(axis=2)            # [n][r]: the group's queries summed
+    if reduce == "sum":
+        return per_key.sum(axis=1)
+    if reduce == "max":
+        return per_key.max(axis=1)
+    raise ValueError(reduce)
 
 
 def score_cosine(rq: np.ndarray, M: np.ndarray) -> np.ndarray:
@@ -260,7 +267,7 @@ def merge_partials(parts):
 
 
 def decode(q, K, V, reps, *, dtype, block_size, sink, window, top_k_blocks,
-           scale=None):
+           scale=None, score_reduce="sum"):
     """One decode step for every (batch, q head).
 
     q [B][Hq][D], K, V [B][Hkv][T][D] as stored (``dtype``, widened here one
@@ -293,7 +300,7 @@ def decode(q, K, V, reps, *, dtype, block_size, sink, window, top_k_blocks,
                 R = widen(K[b, h, cand], dtype)[:, None, :]
             else:
                 R = reps[b, h, cand]
-            s = score_dot(qg, R) if nc else np.zeros(0)
+            s = score_dot(qg, R, score_reduce) if nc else np.zeros(0)
             scores[b, h] = s
             sel = cand[top_k(s, top_k_blocks)]
             idx[b, h] = sel

@@ -193,6 +193,32 @@ def test_score_dot_basis_closed_form():
     np.testing.assert_allclose(O.score_dot(qs, reps), expect, atol=1e-12)
 
 
+def test_score_dot_max_variant_closed_form():
+    # the same basis keys: the max variant takes, per block, the largest of its
+    # r keys' group-summed dot products (not their sum)
+    D, n, r, m = 12, 7, 3, 4
+    rng = _rng(11)
+    qs = rng.normal(size=(m, D))
+    dsel = rng.integers(0, D, size=(n, r))
+    c = rng.normal(size=(n, r))
+    reps = np.zeros((n, r, D))
+    for j in range(n):
+        for i in range(r):
+            reps[j, i, dsel[j, i]] = c[j, i]
+    expect = [max(sum(c[j, i] * qs[q, dsel[j, i]] for q in range(m)) for i in range(r))
+              for j in range(n)]
+    np.testing.assert_allclose(O.score_dot(qs, reps, "max"), expect, atol=1e-12)
+    # one key per block: max and sum agree; the order of the keys does not matter
+    np.testing.assert_allclose(O.score_dot(qs, reps[:, :1], "max"), O.score_dot(qs, reps[:, :1]))
+    perm = reps[:, ::-1]
+    np.testing.assert_allclose(O.score_dot(qs, perm, "max"), O.score_dot(qs, reps, "max"))
+    # a block whose keys are all equal scores max = sum / r
+    same = np.repeat(reps[:, :1], r, axis=1)
+    np.testing.assert_allclose(O.score_dot(qs, same, "max") * r, O.score_dot(qs, same), atol=1e-12)
+    with pytest.raises(ValueError):
+        O.score_dot(qs, reps, "mean")
+
+
 def test_decode_gqa_grouping_closed_form():
     # q head i = (i+1) u, every rep key = u: kv head h sums q heads h*g..h*g+g-1
     B, Hq, Hkv, D, T, bs = 1, 8, 2, 4, 32, 4
