@@ -550,10 +550,11 @@ def _time_graph(g, stream, seconds, min_iters=5):
     return e0.elapsed_time(e1) / n, n
 
 
-def measure_decode_config(name, dev, seconds, pk):
+def measure_decode_config(name, dev, seconds, pk, score_reduce="sum"):
     """Decode-step throughput of one decode config (graph-replayed steps; L2
     defeated by rotating store replicas, or by an L2-sized write between
-    steps whose own time is subtracted when replicas would not fit)."""
+    steps whose own time is subtracted when replicas would not fit).
+    score_reduce="max": the max-over-representative-keys score variant."""
     import torch
     import retrieval_block_sparse_b200 as rba
     from retrieval_block_sparse_b200 import synth
@@ -563,7 +564,8 @@ def measure_decode_config(name, dev, seconds, pk):
     def new_store():
         return rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                          head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
-                         dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep, device=dev)
+                         dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep, device=dev,
+                         score_reduce=score_reduce)
     st = new_store()
     st.k.copy_(_to_dev(x["K"], w.dtype, dev))
     st.v.copy_(_to_dev(x["V"], w.dtype, dev))
@@ -634,7 +636,8 @@ def measure_decode_config(name, dev, seconds, pk):
     us = ms * 1e3
     gbs = nbytes / (us * 1e-6) / 1e9
     plan = st.decode_plan(w.top_k, w.context, w.sink, w.window)
-    return {"workload": name, "steps_per_s": round(1e6 / us, 2), "us_per_step": round(us, 3),
+    return {"workload": name, "score_reduce": score_reduce,
+            "steps_per_s": round(1e6 / us, 2), "us_per_step": round(us, 3),
             "algorithmic_bytes": nbytes, "rep_key_bytes": rep_b, "gathered_kv_bytes": gath_b,
             "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
             "path": {1: "pipelined, persistent attention (CUDA cores)",
@@ -803,6 +806,8 @@ def measure_configs(dev, seconds):
     out = {}
     for name in ("tiny-decode-f32", "landmark-decode-b16", "token-retrieval-decode-1m"):
         out[name] = measure_decode_config(name, dev, seconds, pk)
+    out["infllm-decode-128k:max-over-rep-keys"] = measure_decode_config(
+        "infllm-decode-128k", dev, seconds, pk, score_reduce="max")
     for name in ("memlong-cosine-prefill", "token-retrieval-prefill-1m"):
         out[name] = measure_prefill_config(name, dev, seconds, pk)
     for name in ("memlong-cosine-prefill", "infllm-decode-128k"):

@@ -96,6 +96,13 @@ typedef struct {
   rba_rep_mode mode;
 } rba_store_desc;
 
+/* How the dot-product modes combine a block's n_rep representative keys into one
+ * score (rba_store_set_score_reduce). */
+typedef enum {
+  RBA_SCORE_SUM = 0,  /* default: sum over the keys of the group-summed dot products */
+  RBA_SCORE_MAX = 1   /* variant: the largest of the keys' group-summed dot products */
+} rba_score_reduce;
+
 /* Opaque: host-side description of caller-owned device pools. */
 typedef struct rba_store rba_store;
 
@@ -111,6 +118,14 @@ rba_status rba_store_create(const rba_store_desc* desc, void* k_pool, void* v_po
                             void* rep_pool, int32_t* rep_pos, int32_t* status_word,
                             rba_store** out);
 rba_status rba_store_destroy(rba_store* store);
+
+/* Block-score variant of a store (host only; the default is RBA_SCORE_SUM).  With
+ * RBA_SCORE_MAX, rba_score, rba_decode_step and rba_stream_step score candidate j as
+ * max over the block's keys i of sum over the scoring q rows of q . rep_{j,i}: a block
+ * as relevant as its most relevant representative token ([IL] method: units are
+ * represented by their most-attended tokens; this reading weighs the best one alone).
+ * Errors: INVALID_ARG (unknown value; RBA_SCORE_MAX on cosine or identity stores). */
+rba_status rba_store_set_score_reduce(rba_store* store, int32_t reduce);
 
 /* Candidate range for a store holding T tokens with the given sink/window
  * (host only; see the vocabulary above).  Errors: INVALID_ARG (tail block
@@ -141,7 +156,8 @@ rba_status rba_memorize(rba_store* store, const void* k_src, const void* v_src,
  * [IL] relevance against representative tokens).
  *   dot modes: q device dtype [B][Hq][n_q][D]; for candidate c of (b, kv head h)
  *     scores[b][h][c] = sum over the group's q heads, over the n_q rows, and over the
- *     block's n_rep keys of q . rep  (n_q > 1: a prefill chunk shares one selection)
+ *     block's n_rep keys of q . rep  (n_q > 1: a prefill chunk shares one selection);
+ *     with RBA_SCORE_MAX the sum over the keys becomes a max
  *   cosine mode: q = query embeddings, device fp32 [n_q][d_ret]; store batch must be 1;
  *     scores[i][c] = cos(q_i, M_{first_cand + c})
  *   scores  device fp32 [B][Hkv][nc] (dot) or [n_q][nc] (cosine)

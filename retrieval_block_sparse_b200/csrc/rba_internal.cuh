@@ -17,6 +17,7 @@ struct rba_store {
   int32_t* rep_pos;
   int32_t* status;
   int64_t cap_blocks;
+  int32_t score_reduce;   // rba_score_reduce: how a block's r representative keys combine
 };
 
 namespace rba {

@@ -123,6 +123,7 @@ rba_status launch_score_dot(const rba_store* st, const void* q, int n_q, const f
   a.n_q = n_q;
   a.first = g.first;
   a.nc = g.nc;
+  a.max_over_keys = st->score_reduce == RBA_SCORE_MAX;
   if (d.mode == RBA_REP_IDENTITY) {
     a.rep = st->k;
     a.rep_rows = d.capacity_tokens;

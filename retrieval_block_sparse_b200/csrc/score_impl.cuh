@@ -12,13 +12,14 @@ struct ScoreArgs {
   const float* qsum;    // [B*Hkv][D] or nullptr
   float* scores;        // [B*Hkv][nc]
   int Hq, Hkv, n_q, first, nc;
+  bool max_over_keys;   // block score = max over its keys (else their sum)
 };
 
 // One CTA covers `cand_per_cta` consecutive candidates of one (b, kv head).
 // A candidate's R*D rep elements are contiguous; LPC lanes share one
 // candidate, each loading VPL 16-byte vectors, and U candidate groups are in
 // flight per warp before any arithmetic.
-template <typename QT, typename RT, int D, int R, int NW, int U>
+template <typename QT, typename RT, int D, int R, int NW, int U, bool MAXR>
 __global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int cand_per_cta) {
   constexpr int EPV = Elem<RT>::kPerVec;
   constexpr int VPC = R * D / EPV;
@@ -79,23 +80,61 @@ __global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int can
     if (c0 != c_first) load_groups(c0);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      float acc = 0.f;
+      float part[VPL];  // this lane's share of the dot product, per loaded vector
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
         float f[EPV];
         unpack(v[u][i], f, RT());
+        float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < EPV; ++e) acc = fmaf(qr[i][e], f[e], acc);
+        part[i] = acc;
       }
+      float acc;
+      if constexpr (!MAXR) {
+        acc = 0.f;
 #pragma unroll
-      for (int o = LPC / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        for (int i = 0; i < VPL; ++i) acc += part[i];
+#pragma unroll
+        for (int o = LPC / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      } else {
+        // vector (sub + i LPC) of the candidate belongs to key (sub + i LPC) / VPR
+        constexpr int VPR = D / EPV;  // vectors per representative key
+        if constexpr (VPR >= LPC) {
+          // a key spans VPR / LPC whole vector slots of every lane
+          constexpr int SPK = VPR / LPC;
+          acc = -INFINITY;
+#pragma unroll
+          for (int r0 = 0; r0 < VPL; r0 += SPK) {
+            float kd = 0.f;
+#pragma unroll
+            for (int i = r0; i < r0 + SPK; ++i) kd += part[i];
+#pragma unroll
+            for (int o = LPC / 2; o > 0; o >>= 1) kd += __shfl_xor_sync(0xffffffffu, kd, o);
+            acc = fmaxf(acc, kd);
+          }
+        } else {
+          // a key spans VPR lanes of one vector slot: sum inside those lane
+          // segments, then the max over slots and segments
+          acc = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) {
+            float kd = part[i];
+#pragma unroll
+            for (int o = VPR / 2; o > 0; o >>= 1) kd += __shfl_xor_sync(0xffffffffu, kd, o);
+            acc = fmaxf(acc, kd);
+          }
+#pragma unroll
+          for (int o = VPR; o < LPC; o <<= 1) acc = fmaxf(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+        }
+      }
       const int c = c0 + u * CPW + slot;
       if (sub == 0 && c < c_end) out[c] = acc;
     }
   }
 }
 
-template <typename QT, typename RT, int D, int R>
+template <typename QT, typename RT, int D, int R, bool MAXR>
 rba_status launch_score_dot_t(const ScoreArgs& a, int BH, cudaStream_t stream) {
   constexpr int NW = 8, U = 4;
   constexpr int EPV = Elem<RT>::kPerVec;
@@ -107,7 +146,7 @@ rba_status launch_score_dot_t(const ScoreArgs& a, int BH, cudaStream_t stream) {
   per_cta = (per_cta + per_iter - 1) / per_iter * per_iter;
   if (per_cta < per_iter) per_cta = per_iter;
   const int gx = static_cast<int>((a.nc + per_cta - 1) / per_cta);
-  score_dot_kernel<QT, RT, D, R, NW, U>
+  score_dot_kernel<QT, RT, D, R, NW, U, MAXR>
       <<<dim3(gx, BH), NW * 32, 0, stream>>>(a, static_cast<int>(per_cta));
   RBA_LAUNCH_CHECK();
   return RBA_OK;
@@ -115,11 +154,20 @@ rba_status launch_score_dot_t(const ScoreArgs& a, int BH, cudaStream_t stream) {
 
 template <typename QT, typename RT, int D>
 rba_status dispatch_r(const ScoreArgs& a, int R, int BH, cudaStream_t s) {
+  // with one key per block the max over keys is the sum
+  if (a.max_over_keys && R > 1) {
+    switch (R) {
+      case 2: return launch_score_dot_t<QT, RT, D, 2, true>(a, BH, s);
+      case 4: return launch_score_dot_t<QT, RT, D, 4, true>(a, BH, s);
+      case 8: return launch_score_dot_t<QT, RT, D, 8, true>(a, BH, s);
+    }
+    return RBA_ERR_UNSUPPORTED;
+  }
   switch (R) {
-    case 1: return launch_score_dot_t<QT, RT, D, 1>(a, BH, s);
-    case 2: return launch_score_dot_t<QT, RT, D, 2>(a, BH, s);
-    case 4: return launch_score_dot_t<QT, RT, D, 4>(a, BH, s);
-    case 8: return launch_score_dot_t<QT, RT, D, 8>(a, BH, s);
+    case 1: return launch_score_dot_t<QT, RT, D, 1, false>(a, BH, s);
+    case 2: return launch_score_dot_t<QT, RT, D, 2, false>(a, BH, s);
+    case 4: return launch_score_dot_t<QT, RT, D, 4, false>(a, BH, s);
+    case 8: return launch_score_dot_t<QT, RT, D, 8, false>(a, BH, s);
   }
   return RBA_ERR_UNSUPPORTED;
 }

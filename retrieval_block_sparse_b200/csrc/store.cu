@@ -108,6 +108,7 @@ rba_status rba_store_create(const rba_store_desc* d, void* k_pool, void* v_pool,
   s->rep_pos = rep_pos;
   s->status = status_word;
   s->cap_blocks = d->capacity_tokens / d->block_size;
+  s->score_reduce = RBA_SCORE_SUM;
   *out = s;
   return RBA_OK;
 }
@@ -157,3 +158,13 @@ const char* rba_status_string(rba_status s) {
 int32_t rba_version(void) { return 100; }
 
 }  // extern "C"
+
+extern "C" rba_status rba_store_set_score_reduce(rba_store* st, int32_t reduce) {
+  if (st == nullptr || (reduce != RBA_SCORE_SUM && reduce != RBA_SCORE_MAX))
+    return RBA_ERR_INVALID_ARG;
+  if (reduce == RBA_SCORE_MAX && (st->d.mode == RBA_REP_EMBED_COSINE ||
+                                  st->d.mode == RBA_REP_IDENTITY))
+    return RBA_ERR_INVALID_ARG;
+  st->score_reduce = reduce;
+  return RBA_OK;
+}

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(PKG, "librba.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(7)
 F32, BF16 = 0, 1
 MODES = {"mean": 0, "topr_attn": 1, "external": 2, "embed_cosine": 3, "identity": 4}
+SCORE_REDUCE = {"sum": 0, "max": 1}
 
 _c_i32, _c_i64, _c_f32, _c_size, _p = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
                                         ctypes.c_size_t, ctypes.c_void_p)
@@ -26,6 +27,7 @@ _c_i32, _c_i64, _c_f32, _c_size, _p = (ctypes.c_int32, ctypes.c_int64, ctypes.c_
 SIGNATURES = {
     "rba_store_create": (_c_i32, [_p, _p, _p, _p, _p, _p, ctypes.POINTER(_p)]),
     "rba_store_destroy": (_c_i32, [_p]),
+    "rba_store_set_score_reduce": (_c_i32, [_p, _c_i32]),
     "rba_candidates": (_c_i32, [_p, _c_i64, _c_i32, _c_i32, ctypes.POINTER(_c_i32),
                                 ctypes.POINTER(_c_i32)]),
     "rba_memorize": (_c_i32, [_p, _p, _p, _c_i64, _c_i32, _p, _c_i32, _c_f32, _p]),
@@ -131,10 +133,12 @@ class Store:
                [B][cap_blocks][d_ret]; identity: none
       rep_pos  int32 [B][Hkv][cap_blocks][r] (topr_attn)
       status   int32[4] device status word
+    score_reduce: "sum" (default) or "max" -- how a block's r representative
+    keys combine into its score (rba_store_set_score_reduce).
     """
 
     def __init__(self, *, batch, n_q_heads, n_kv_heads, head_dim, block_size, capacity_tokens,
-                 dtype="bf16", mode="mean", n_rep=1, d_ret=0, device="cuda"):
+                 dtype="bf16", mode="mean", n_rep=1, d_ret=0, device="cuda", score_reduce="sum"):
         self.dtype = BF16 if dtype in ("bf16", torch.bfloat16) else F32
         self.mode = mode
         self.B, self.Hq, self.Hkv, self.D = batch, n_q_heads, n_kv_heads, head_dim
@@ -167,6 +171,10 @@ class Store:
                                       _ptr(self.rep_pos), _ptr(self.status), ctypes.byref(h)),
                "rba_store_create")
         self.handle = h
+        if score_reduce != "sum":
+            _check(lib().rba_store_set_score_reduce(h, SCORE_REDUCE[score_reduce]),
+                   "rba_store_set_score_reduce")
+        self.score_reduce = score_reduce
 
     def __del__(self):
         h = getattr(self, "handle", None)

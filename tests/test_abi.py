@@ -166,3 +166,15 @@ def test_memory_update_argument_checks_launch_nothing(L):
     assert L.rba_count_retrievals(h, FAKE, 2, 0, FAKE, None) == 0
     assert L.rba_count_retrievals(h, FAKE, 2, 4, None, None) == 1
     L.rba_store_destroy(h)
+
+
+def test_score_reduce_setter_checks(L):
+    s, h = _create(L, mode=1, n_rep=4)                  # top-r keys
+    assert L.rba_store_set_score_reduce(h, 1) == 0
+    assert L.rba_store_set_score_reduce(h, 0) == 0
+    assert L.rba_store_set_score_reduce(h, 2) == 1      # unknown value
+    L.rba_store_destroy(h)
+    s, h = _create(L, mode=4, block_size=1)             # identity: nothing to reduce
+    assert L.rba_store_set_score_reduce(h, 1) == 1
+    L.rba_store_destroy(h)
+    assert L.rba_store_set_score_reduce(None, 1) == 1
