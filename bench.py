@@ -30,6 +30,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import sys
 import threading
 import time
@@ -107,11 +108,19 @@ def peaks():
     return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def _code_only(text):
+    """Source text without comments and blank space: edits to comments do not
+    change a kernel, so they do not invalidate its recorded counters."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash(kernel):
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "retrieval_block_sparse_b200", rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "retrieval_block_sparse_b200", rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

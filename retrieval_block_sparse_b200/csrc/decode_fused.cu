@@ -6,19 +6,23 @@
 // window, one state per q head, log-sum-exp merge of partial states).  The
 // decode step launches three kernels back to back -- block scores, top-k,
 // this kernel -- the last two as programmatic dependents, so this kernel
-// starts while the selection is still running:
-//   * one CTA per SM (minus the SMs the top-k kernel holds): warp 0 stages,
-//     warps 1..7 compute;
-//   * every CTA gets an equal share of the flattened attention list; a
-//     head's share mixes sink + window rows (known without the selection)
-//     and rows of the selected blocks in proportion, sink/window first;
-//   * warp 0 walks the same item sequence as the compute warps and stages
-//     each item with bulk asynchronous copies (whole contiguous runs of K/V
-//     rows) into a ring of shared-memory stages guarded by full / empty
-//     mbarriers; before the first selected row it waits for the top-k
-//     kernel to complete (griddepcontrol.wait);
-//   * partial softmax states go to per-(head, CTA) slots; the last
-//     contributor of a head merges them (no CTA waits for another).
+// starts while the selection is still running.  Two kernels share the work
+// list, the staging scheme and the end-of-head merge:
+//   * decode_mma_kernel (bf16 stores whose blocks are whole 64-row tiles):
+//     the staging warp loads single-segment pieces of up to 64 rows as
+//     swizzled 2-D tensor boxes; eight compute warps run the inner products
+//     on the tensor cores (mma.sync), two pieces at a time;
+//   * decode_fused_kernel (other block sizes, fp32): the staging warp copies
+//     whole contiguous runs of K/V rows into 56-row tiles; fourteen compute
+//     warps run the online softmax on the CUDA cores.
+// In both, one CTA runs per SM (minus the SMs the top-k kernel holds); every
+// CTA gets an equal share of the flattened attention list, and a head's share
+// mixes sink + window rows (known without the selection) and rows of the
+// selected blocks in proportion, sink/window first.  The staging warp fills a
+// ring of shared-memory stages guarded by full / empty mbarriers and waits
+// for the top-k kernel (griddepcontrol.wait) only before the first selected
+// row.  Partial softmax states go to per-(head, CTA) slots; the last
+// contributor of a head merges them (no CTA waits for another).
 // All mbarrier waits are bounded in time; on expiry the kernel records
 // RBA_ERR_TIMEOUT in the status word, skips the remaining work, waits
 // (bounded) for its copies in flight and terminates.
