@@ -52,6 +52,7 @@ struct PrefillArgs {
   int store_batch;     // 1 (one memory for all chunks) or n_chunks
   int staged;          // past tokens come from the staging buffer
   int n_att_max;       // staging rows per (chunk, kv head)
+  int pairs_outer;     // grid order: 1 = (head, chunk, pair), heaviest pairs first
   float scale_log2;
 };
 
@@ -314,7 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   int4* tiles = reinterpret_cast<int4*>(smem + kTileOff);
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int pt = blockIdx.x, hq = blockIdx.y, c = blockIdx.z;
+  // grid order.  Many pairs per chunk (their causal work differs a lot): the
+  // slowest index runs over the query-tile pairs, later (heavier) pairs first,
+  // so the last partial wave holds light CTAs.  Else the pairs of one (head,
+  // chunk) are neighbours and share its retrieved K/V in L2.
+  const int pt = a.pairs_outer ? gridDim.z - 1 - blockIdx.z : blockIdx.x;
+  const int hq = a.pairs_outer ? blockIdx.x : blockIdx.y;
+  const int c = a.pairs_outer ? blockIdx.y : blockIdx.z;
   const int h = hq / a.G;
   // query tiles of this CTA: X = 0 (A) rows [256 pt, +128), X = 1 (B) the next 128
   const int qt0 = 2 * pt;
@@ -791,8 +798,13 @@ rba_status rba_attend_prefill(const rba_store* st, const void* q, int32_t n_chun
     msv = mpv;
   }
   RBA_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(prefill_kernel), kSmemBytes));
-  const dim3 grid(static_cast<unsigned>((chunk_len + 2 * kBM - 1) / (2 * kBM)),
-                  static_cast<unsigned>(d.n_q_heads), static_cast<unsigned>(n_chunks));
+  const unsigned n_pairs = static_cast<unsigned>((chunk_len + 2 * kBM - 1) / (2 * kBM));
+  a.pairs_outer = n_pairs > 2 ? 1 : 0;
+  const dim3 grid = a.pairs_outer
+                        ? dim3(static_cast<unsigned>(d.n_q_heads),
+                               static_cast<unsigned>(n_chunks), n_pairs)
+                        : dim3(n_pairs, static_cast<unsigned>(d.n_q_heads),
+                               static_cast<unsigned>(n_chunks));
   prefill_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a, mq, mpk, mpv, msk, msv, mck, mcv);
   RBA_LAUNCH_CHECK();
   return RBA_OK;
