@@ -13,5 +13,7 @@ from .retrieval import *  # noqa: F401,F403
 from .retrieval import __all__ as _r_all
 from .memory import *  # noqa: F401,F403
 from .memory import __all__ as _m_all
+from .approx import *  # noqa: F401,F403
+from .approx import __all__ as _a_all
 
-__all__ = list(_r_all) + list(_m_all)
+__all__ = list(_r_all) + list(_m_all) + list(_a_all)

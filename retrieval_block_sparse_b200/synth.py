@@ -212,6 +212,9 @@ def decode_inputs(w: DecodeWorkload) -> dict:
       landmark  q, K, V, landmark keys ~ N(0, 1); per (batch, head) one block
                 j* before the window is drawn and q = 0.5 L[j*] + sqrt(0.75) z.
       shifted   K, V ~ N(0, 1); q ~ N(0.5, 1.5^2) (query/key distribution gap).
+      drift     as shifted, but each key channel drifts slowly along the sequence
+                (first-order autoregression, correlation 0.97 between neighbouring
+                tokens, unit variance): nearby keys resemble each other.
     """
     B, Hq, Hkv, D, T, bs = (w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
                             w.context, w.block_size)
@@ -225,6 +228,16 @@ def decode_inputs(w: DecodeWorkload) -> dict:
     if w.recipe == "normal":
         q = _normal(s, "q", (B, Hq, D))
     elif w.recipe == "shifted":
+        q = _normal(s, "q", (B, Hq, D), mean=0.5, std=1.5)
+    elif w.recipe == "drift":
+        from scipy.signal import lfilter
+        rho = 0.97
+        for b in range(B):
+            for h in range(Hkv):
+                z = K[b, h]
+                zi = (rho * z[0])[None, :]
+                K[b, h, 1:] = lfilter([math.sqrt(1.0 - rho * rho)], [1.0, -rho], z[1:], axis=0,
+                                      zi=zi)[0]
         q = _normal(s, "q", (B, Hq, D), mean=0.5, std=1.5)
     elif w.recipe == "planted":
         u = _unit_rows(_normal(s, "u", (Hkv, D)).astype(np.float64)).astype(np.float32)
