@@ -5,9 +5,11 @@ tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
 import it.  It shares no code with the CUDA path; both read the same seeded
 inputs from ``retrieval_block_sparse_b200.synth`` and nothing else.
 
-Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
-invariants, library routines or brute force; see the docstring of each
-function for the passage of the pages it restates.
+Every function is pinned against closed forms, invariants, library routines
+or brute force: ``tests/test_oracle_pins.py`` (retrieval attention),
+``tests/test_oracle_memory_pins.py`` (dynamic memory update) and
+``tests/test_oracle_approx_pins.py`` (two-stage approximate retrieval); see
+the docstring of each function for the passage of the pages it restates.
 """
 from .retrieval import *  # noqa: F401,F403
 from .retrieval import __all__ as _r_all

@@ -99,3 +99,12 @@ def test_prefill_pairs_match_brute_force_and_published_sizes():
     c5 = W["token-retrieval-prefill-1m"]
     idx5 = np.tile(np.arange(128, 128 + 2048), (1, c5.n_kv_heads, 1))
     assert bench.prefill_pairs(c5, idx5) == 32 * (2048 * 2688 + 2048 * 2049 // 2)
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    import bench
+    code = "int f(int x) {\n  return x + 1;  // one more\n}\n/* block\n comment */\n"
+    same = "// header\nint f(int x) {\n  return x + 1;\n}\n"
+    other = "int f(int x) {\n  return x + 2;\n}\n"
+    assert bench._code_only(code) == bench._code_only(same)
+    assert bench._code_only(code) != bench._code_only(other)
