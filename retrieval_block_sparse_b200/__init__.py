@@ -3,7 +3,10 @@
 Context-memory retrieval attention for long-context decode and chunked
 prefill: blocks of past K/V are scored by representative keys or embeddings,
 the top-k blocks per KV head are selected, and exact softmax attention runs
-over sink tokens, retrieved blocks and the local window.
+over sink tokens, retrieved blocks and the local window.  Around that path:
+a streaming decode step (append a token, memorise the block it completes,
+decode), counter-driven dynamic memory update with in-place compaction, and
+a max-over-representative-keys score variant.
 
 All computation is in the CUDA library ``librba.so`` (C ABI:
 ``include/rba.h``); ``rba`` is its Python binding.  ``synth`` draws the seeded
