@@ -6,8 +6,8 @@ Source: RetrievalAttention summary (arXiv 2409.10516), "proposed method": the
 attention of a query is computed over the few keys that matter, found by an
 approximate nearest-neighbour search instead of a scan of every key, and a
 search adapted to the query/key distribution gap reads only 1-3% of the
-keys.  The page names no index structure; the reading taken here (listed in
-the design notes) is the plainest one that the rest supports:
+keys.  The page names no index structure; the reading taken here is the
+plainest one that the rest supports:
 
   * index: consecutive groups of c candidate tokens (the blocks of size c of
     the candidate rule), each represented by the mean of its keys;

@@ -9,7 +9,7 @@ counters of how often each entry was retrieved decide what stays.  The newest
 dropped (likely stale), and in the middle 80% the least retrieved entries are
 deleted until the memory holds 50% of what it held.
 
-Readings taken where the page is silent (each listed in the design notes):
+Readings taken where the page is silent:
   * an entry is one block of the store (one token when the block size is 1);
     the update runs per memory unit: per (batch, kv head) for the dot-product
     modes, per batch row for the cosine bank, whose K/V of every kv head

@@ -24,7 +24,7 @@ Sources (pages, by title and section):
   [RA]  RetrievalAttention summary (arXiv 2409.10516), "proposed method":
         token-level retrieval (every key its own unit) by vector search.
 
-Readings taken where the pages are silent (each listed in the design notes):
+Readings taken where the pages are silent:
   * candidate rule: a block is scored iff it is a full block with at least one
     token in [sink, T - window);
   * attended set: sink U retrieved blocks U window as a set (each token once);

@@ -7,7 +7,9 @@ Tolerances (stated by the method's accuracy target):
     <= 2e-3 for bf16 inputs, 1e-5 for fp32 inputs;
   * selections: bit-exact, except where the oracle's k-th and (k+1)-th scores
     differ by less than 1e-5 relative -- there either choice is accepted, and
-    only indices inside that near-tie may differ;
+    only indices inside that near-tie may differ; the outputs of such a unit
+    are compared with the oracle evaluated on the GPU's own selection, so
+    every unit is checked against the oracle;
   * scores (no stated bound; derived from fp32 accumulation of n products):
     |s_gpu - s_ref| <= 1e-5 * sum |products|, about 10x the expected fp32
     rounding of an n <= 2048 term dot product.
@@ -113,3 +115,41 @@ def score_tolerance(qsum_abs, reps_abs):
 
 def scale_of(w):
     return 1.0 / math.sqrt(w.head_dim)
+
+
+def check_decode_step(w, q, K, V, ref, idx, out, lse, *, T=None, k=None, min_exact=0.9):
+    """Acceptance of a whole decode step against the oracle, per (b, kv head).
+
+    The GPU selection idx[b, h] must equal the oracle's, or be an accepted
+    near-tie swap (selection_check).  Every q head's output and lse are then
+    compared with the oracle's attention over the GPU-chosen token set: for an
+    exact selection that is ref["out"] / ref["lse"]; for a near-tie swap the
+    oracle's softmax_attention is evaluated on the attended tokens of the
+    GPU's blocks.  q, K, V: the stored inputs (numpy, store dtype bits).
+    Returns the number of units whose selection matched exactly; at least
+    min_exact of them must (near-ties are rare on these inputs)."""
+    T = w.context if T is None else T
+    k = w.top_k if k is None else k
+    g = w.n_q_heads // w.n_kv_heads
+    scale = scale_of(w)
+    tol = OUT_TOL[w.dtype]
+    first = int(ref["cand"][0]) if ref["cand"].size else 0
+    exact = 0
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            kind = selection_check(ref["scores"][b, h], k, first, idx[b, h])
+            toks = O.attended_tokens(T, w.block_size, w.sink, w.window, idx[b, h])
+            Kt = O.widen(K[b, h, toks], w.dtype)
+            Vt = O.widen(V[b, h, toks], w.dtype)
+            for i in range(h * g, (h + 1) * g):
+                if kind == "exact":
+                    o_ref, l_ref = ref["out"][b, i], ref["lse"][b, i]
+                else:
+                    o_ref, l_ref, _ = O.softmax_attention(O.widen(q[b, i], w.dtype), Kt, Vt,
+                                                          scale)
+                err = out_error(out[b, i], o_ref, Vt)
+                assert err <= tol, (b, h, i, kind, err)
+                assert abs(lse[b, i] - l_ref) <= tol, (b, h, i, kind, lse[b, i], l_ref)
+            exact += kind == "exact"
+    assert exact >= min_exact * w.batch * w.n_kv_heads
+    return exact

@@ -4,7 +4,8 @@ attention) against the fp64 oracle, through the C ABI.
 Selections are computed on the GPU (rba_score + rba_topk) and checked against
 the oracle's; the attention is then run on the oracle's selection so that
 outputs are compared on identical token sets.  Full-size workloads compare a
-seeded sample of query rows and heads (the oracle walks rows one by one)."""
+seeded sample of query rows (24 random rows plus the first and last row of
+every 128-row tile) and heads (the oracle walks rows one by one)."""
 import numpy as np
 import pytest
 import torch
@@ -68,7 +69,10 @@ def _run(rba, name):
     rng = np.random.default_rng(7)
     rows = heads = None
     if name in FULL:
-        rows = sorted(rng.choice(w.chunk_len, 24, replace=False).tolist())
+        # 24 random rows plus the first and last row of every 128-row query
+        # tile (the tile edges and the causal diagonal's ends)
+        edges = {r for t in range(0, w.chunk_len, 128) for r in (t, t + 127) if r < w.chunk_len}
+        rows = sorted(set(rng.choice(w.chunk_len, 24, replace=False).tolist()) | edges)
         heads = sorted(rng.choice(w.n_q_heads, 3, replace=False).tolist())
     ref = O.prefill(x["Q"], x["K"], x["V"], x["chunk_K"], x["chunk_V"], dtype="bf16",
                     block_size=w.block_size, sink=w.sink, window=w.window,

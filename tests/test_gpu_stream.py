@@ -15,7 +15,7 @@ import torch
 import oracle as O
 from retrieval_block_sparse_b200 import synth
 
-from parity import OUT_TOL, attended_v_max, dev, out_error, selection_check
+from parity import check_decode_step, dev
 
 pytestmark = pytest.mark.gpu
 W = synth.WORKLOADS
@@ -70,7 +70,6 @@ def test_stream_steps_match_oracle(rba, name):
                 aux=(aux_all[:, :, :nb0].contiguous() if w.rep_mode == "external" else aux_all))
     rng = np.random.default_rng(w.seed)
     ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)
-    g = w.n_q_heads // w.n_kv_heads
     checked = 0
     for i in range(STEPS):
         T = T0 + i
@@ -93,17 +92,8 @@ def test_stream_steps_match_oracle(rba, name):
         assert idx.shape[-1] == ke
         ref = O.decode(qn, x["K"][:, :, :Tn], x["V"][:, :, :Tn], _reps(w, x, Tn), dtype=w.dtype,
                        block_size=w.block_size, sink=w.sink, window=w.window, top_k_blocks=ke)
-        idx_h, out_h, lse_h = idx.cpu().numpy(), out.cpu().numpy(), lse.cpu().numpy()
-        xs = dict(x, K=x["K"][:, :, :Tn], V=x["V"][:, :, :Tn])
-        ws_ = w.scaled(context=Tn)
-        for b in range(w.batch):
-            for h in range(w.n_kv_heads):
-                kind = selection_check(ref["scores"][b, h], ke, first, idx_h[b, h])
-                va = attended_v_max(ws_, xs, b, h, idx_h[b, h])
-                for qh in range(h * g, (h + 1) * g):
-                    if kind == "exact":
-                        assert out_error(out_h[b, qh], ref["out"][b, qh], va) <= OUT_TOL[w.dtype]
-                        assert abs(lse_h[b, qh] - ref["lse"][b, qh]) <= OUT_TOL[w.dtype]
+        check_decode_step(w, qn, x["K"], x["V"], ref, idx.cpu().numpy(), out.cpu().numpy(),
+                          lse.cpu().numpy(), T=Tn, k=ke)
     assert checked >= 6
 
 

@@ -394,6 +394,88 @@ def test_prefill_dot_scores_are_chunk_summed_query():
     np.testing.assert_allclose(res["scores"][0, 0], expect, atol=1e-12)
 
 
+def _cosine_prefill_case(seed):
+    """Memory of 10 blocks of 4 tokens, sink 6, window 10: block 0 lies in the
+    sink, blocks 8 and 9 in the window, so the candidates are blocks 1..7 and
+    candidate c is block c + 1 (a non-zero candidate offset).  Bank entry j is
+    the one-hot vector e_j (orthogonal entries: cosines are closed forms)."""
+    Hq, Hkv, D, T, bs, Nq, S, W = 4, 2, 8, 40, 4, 3, 6, 10
+    rng = _rng(seed)
+    Q = rng.normal(size=(2, Hq, Nq, D)).astype(np.float32)
+    K = rng.normal(size=(1, Hkv, T, D)).astype(np.float32)
+    V = rng.normal(size=(1, Hkv, T, D)).astype(np.float32)
+    Kc = rng.normal(size=(2, Hkv, Nq, D)).astype(np.float32)
+    Vc = rng.normal(size=(2, Hkv, Nq, D)).astype(np.float32)
+    bank = np.eye(T // bs)
+    return Q, K, V, Kc, Vc, bank, bs, S, W
+
+
+def test_prefill_cosine_selection_is_shared_and_offset():
+    # MemLong 2.3.2: each query chunk retrieves by cosine(r_q, M_j) over the
+    # memory's candidate blocks, one selection for all heads.  r_q mixes bank
+    # directions with known weights, so the cosines are weight / |r_q|; the
+    # heaviest directions include a sink block (0) and a window block (9),
+    # which are not candidates and must not be selected.
+    Q, K, V, Kc, Vc, bank, bs, S, W = _cosine_prefill_case(18)
+    T, D, Nq = K.shape[2], K.shape[3], Q.shape[2]
+    weights = [{0: 5.0, 2: 3.0, 5: 2.0, 9: 4.0, 6: 0.5},
+               {7: 2.5, 1: 2.0, 9: 6.0, 3: 1.0, 0: 3.0}]
+    expect = [[2, 5], [1, 7]]
+    qe = np.zeros((2, bank.shape[1]))
+    for c, wc in enumerate(weights):
+        for j, a in wc.items():
+            qe[c, j] = a
+    res = O.prefill(Q, K, V, Kc, Vc, dtype="f32", block_size=bs, sink=S, window=W,
+                    top_k_blocks=2, score_mode="cosine", query_embed=qe, bank=bank)
+    np.testing.assert_array_equal(res["cand"], np.arange(1, 8))
+    assert res["idx"].shape == (2, 1, 2)
+    for c in range(2):
+        norm = math.sqrt(sum(a * a for a in weights[c].values()))
+        closed = [weights[c].get(j, 0.0) / norm for j in range(1, 8)]
+        np.testing.assert_allclose(res["scores"][c, 0], closed, atol=1e-15)
+        np.testing.assert_array_equal(res["idx"][c, 0], expect[c])
+        # every q head attends sink U the chunk's selected blocks U window,
+        # then its own chunk causally (torch fp64 attention, explicit mask)
+        toks = sorted(set(range(S)) | set(range(T - W, T)) |
+                      {t for j in expect[c] for t in range(j * bs, (j + 1) * bs)})
+        for hq in range(Q.shape[1]):
+            h = hq // 2
+            Kall = np.concatenate([K[0, h, toks], Kc[c, h]]).astype(np.float64)
+            Vall = np.concatenate([V[0, h, toks], Vc[c, h]]).astype(np.float64)
+            n = len(toks)
+            mask = np.zeros((Nq, n + Nq), dtype=bool)
+            for i in range(Nq):
+                mask[i, :n + i + 1] = True
+            ref = _sdpa(Q[c, hq].astype(np.float64), Kall, Vall, D ** -0.5, mask)
+            np.testing.assert_allclose(res["out"][c, hq], ref, atol=1e-12)
+
+
+def test_prefill_cosine_every_candidate_is_causal_attention():
+    # k = every candidate: sink U blocks 1..7 U window covers all T past
+    # tokens, so every row is causal attention over [past ; chunk], for every
+    # q head, whatever the query embedding
+    Q, K, V, Kc, Vc, bank, bs, S, W = _cosine_prefill_case(19)
+    T, D, Nq = K.shape[2], K.shape[3], Q.shape[2]
+    qe = _rng(20).normal(size=(2, bank.shape[1]))
+    res = O.prefill(Q, K, V, Kc, Vc, dtype="f32", block_size=bs, sink=S, window=W,
+                    top_k_blocks=7, score_mode="cosine", query_embed=qe, bank=bank)
+    mask = np.zeros((Nq, T + Nq), dtype=bool)
+    for i in range(Nq):
+        mask[i, :T + i + 1] = True
+    for c in range(2):
+        np.testing.assert_array_equal(res["idx"][c, 0], np.arange(1, 8))
+        for hq in range(Q.shape[1]):
+            h = hq // 2
+            Kall = np.concatenate([K[0, h], Kc[c, h]]).astype(np.float64)
+            Vall = np.concatenate([V[0, h], Vc[c, h]]).astype(np.float64)
+            full = _sdpa(Q[c, hq].astype(np.float64), Kall, Vall, D ** -0.5, mask)
+            np.testing.assert_allclose(res["out"][c, hq], full, atol=1e-12)
+            lse = scipy.special.logsumexp(
+                np.where(mask, D ** -0.5 * (Kall @ Q[c, hq].astype(np.float64).T).T, -np.inf),
+                axis=1)
+            np.testing.assert_allclose(res["lse"][c, hq], lse, atol=1e-12)
+
+
 # ---------------------------------------------------------------------------
 # retrieval sanity on the synthetic recipes (statistical, not parity)
 
