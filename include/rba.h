@@ -211,8 +211,14 @@ size_t rba_attend_workspace_size(const rba_store* store, int32_t k, int64_t T, i
  * RBA_ATTEND_NOALLOC_SCRATCH_BYTES long, which every GPU that loads the library
  * holds until the process exits.
  *   - Allocates nothing: no cudaMalloc / cudaFree and no allocating library call.
+ *     The array itself is reserved by the CUDA driver when it loads the part of
+ *     the library that holds it on a device: under lazy module loading (the
+ *     default of recent CUDA releases) that happens at the first call on that
+ *     device, otherwise when the library's kernels are loaded.
  *   - The first call on each device looks up the array's device address, with
- *     that device current; make that first call before any stream capture.
+ *     that device current; that lookup may load the module (above), which can
+ *     reserve memory and synchronise.  Make the first call on each device at
+ *     start-up: before any stream capture and outside latency-sensitive paths.
  *   - Each call zeroes the array's ticket region on `stream`, then launches.
  *   - Every call shares the one array, which keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other host threads) race and

@@ -1,4 +1,5 @@
 // Block store description, candidate geometry, status handling.
+#include <atomic>
 #include <mutex>
 #include <new>
 #include <unordered_map>
@@ -31,17 +32,25 @@ rba_status geometry(const rba_store* st, int64_t T, int32_t sink, int32_t window
   return RBA_OK;
 }
 
+// SM count of the current device, cached per device (devices may differ).
 int num_sms() {
-  static int cached = 0;
-  if (cached == 0) {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-      cached = n;
-    else
-      cached = 148;
+  constexpr int kDevices = 64;
+  static std::atomic<int> cached[kDevices];  // 0: not looked up yet
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= kDevices) {
+    int n = 0;
+    return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0
+               ? n
+               : 148;
   }
-  return cached;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
 }
 
 cudaError_t ensure_smem(const void* kernel, size_t bytes) {

@@ -9,7 +9,9 @@ device array inside the library instead.
 This test calls it through the C ABI twice in a row (different queries, the
 second call reusing whatever the first left in the shared array) and checks
 each output against rba_attend's, within the attention tolerance the other
-tests use (2e-3 of max |V| for bf16).  It also checks the size limit.  This
+tests use (2e-3 of max |V| for bf16).  It also checks the size limit: a
+problem whose split-K scratch (computed here from the documented layout) fits
+runs and matches rba_attend, one just over it is rejected.  This
 file is collected last, and it passes on its own in a fresh process too (its
 first call is the first use of the array on the device).
 """
@@ -58,19 +60,45 @@ def test_noalloc_matches_attend_twice(rba):
         assert float((lse - l_ref).abs().max()) <= OUT_TOL[w.dtype]
 
 
-def test_noalloc_rejects_sizes_beyond_the_limit(rba):
-    # 160 x 32 MHA heads: the split partials need more than the fixed array
-    w = synth.WORKLOADS["landmark-decode-b16"].scaled(batch=160, context=100)
+def _split_k_scratch_bytes(batch, n_kv_heads, n_q_heads, head_dim, nsplit):
+    """The split-K kernel's scratch as the library lays it out: merge tickets
+    (one uint32 per (batch, kv head), 256-byte aligned), then one partial state
+    (m, l, o[D]) of fp32 per (batch, q head, split), 256-byte aligned."""
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    return up(4 * batch * n_kv_heads) + up(batch * n_q_heads * nsplit * (head_dim + 2) * 4)
+
+
+@pytest.mark.parametrize("batch,fits", [(125, True), (126, False)])
+def test_noalloc_limit_is_the_split_k_scratch(rba, batch, fits):
+    # 32 MHA heads of 100 tokens per batch row: with more (batch, kv head)
+    # units than SMs and rows this short the split-K kernel uses one split, so
+    # its scratch is 4 B of ticket plus 32 * 130 * 4 B of partials per row:
+    # 125 rows fit in the fixed array, 126 do not
+    w = synth.WORKLOADS["landmark-decode-b16"].scaled(batch=batch, context=100)
+    need = _split_k_scratch_bytes(batch, w.n_kv_heads, w.n_q_heads, w.head_dim, 1)
+    assert (need <= (2 << 20)) == fits
     st = rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                    head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
                    dtype="bf16", mode="external")
-    need = rba.lib().rba_attend_workspace_size(st.handle, 0, w.context, w.sink, w.window)
-    assert need > (2 << 20)
-    q = torch.zeros((w.batch, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(batch)
+    st.k.copy_(torch.randn(st.k.shape, generator=gen, device="cuda").to(torch.bfloat16))
+    st.v.copy_(torch.randn(st.v.shape, generator=gen, device="cuda").to(torch.bfloat16))
+    q = torch.randn((w.batch, w.n_q_heads, w.head_dim), generator=gen,
+                    device="cuda").to(torch.bfloat16)
     idx = torch.zeros((w.batch, w.n_kv_heads, 0), dtype=torch.int32, device="cuda")
-    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), device="cuda")
-    lse = torch.empty((w.batch, w.n_q_heads), device="cuda")
-    assert _noalloc(rba, st, q, idx, w, out, lse) == rba.ERR_WORKSPACE
+    out = torch.full((w.batch, w.n_q_heads, w.head_dim), float("nan"), device="cuda")
+    lse = torch.full((w.batch, w.n_q_heads), float("nan"), device="cuda")
+    s = _noalloc(rba, st, q, idx, w, out, lse)
+    if not fits:
+        assert s == rba.ERR_WORKSPACE
+        assert torch.isnan(out).all()  # nothing launched
+        return
+    assert s == rba.OK
+    st.check()
+    o_ref, l_ref = st.attend(q, idx, w.context, w.sink, w.window)
+    vmax = float(st.v.float().abs().max())
+    assert float((out - o_ref).abs().max()) / vmax <= OUT_TOL["bf16"]
+    assert float((lse - l_ref).abs().max()) <= OUT_TOL["bf16"]
 
 
 SPLIT_K_CASES = {
