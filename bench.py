@@ -49,8 +49,10 @@ KERNEL_SOURCES = {
     "attend_decode_kernel": ["csrc/attend.cu", "csrc/attend_impl.cuh", "csrc/rba_internal.cuh"],
     "decode_fused_kernel": ["csrc/decode_fused.cu", "csrc/attend_impl.cuh",
                             "csrc/rba_internal.cuh"],
-    "decode_mma_kernel": ["csrc/decode_fused.cu", "csrc/attend_impl.cuh",
-                          "csrc/rba_internal.cuh", "csrc/tmap.cu"],
+    "decode_mma_kernel": ["csrc/decode_fused.cu", "csrc/decode_persist.cuh",
+                          "csrc/attend_impl.cuh", "csrc/rba_internal.cuh", "csrc/tmap.cu"],
+    "decode_step_kernel": ["csrc/decode_step.cu", "csrc/decode_persist.cuh",
+                           "csrc/attend_impl.cuh", "csrc/rba_internal.cuh", "csrc/tmap.cu"],
 }
 
 
@@ -118,7 +120,7 @@ def _code_only(text):
 
 def source_hash(kernel):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES[kernel]:
+    for rel in KERNEL_SOURCES.get(kernel, []):
         with open(os.path.join(ROOT, "retrieval_block_sparse_b200", rel), encoding="utf-8") as f:
             h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
@@ -445,8 +447,15 @@ def run_ours(args):
     att_gbs = gath_b / (att_us * 1e-6) / 1e9
     step_us = ms_max * 1e3 / args.steps
     step_gbs = bytes_step / (step_us * 1e-6) / 1e9
-    dom = {1: "decode_fused_kernel", 2: "decode_mma_kernel"}.get(plan, "attend_decode_kernel")
-    dom_bytes, dom_us, dom_gbs = gath_b, att_us, att_gbs
+    if plan == 3:
+        # the whole step is one kernel: its algorithmic bytes over the average
+        # step of the timed region (launch gaps included)
+        dom = "decode_step_kernel"
+        dom_bytes, dom_us, dom_gbs = bytes_step, step_us, step_gbs
+    else:
+        dom = {1: "decode_fused_kernel", 2: "decode_mma_kernel"}.get(plan,
+                                                                     "attend_decode_kernel")
+        dom_bytes, dom_us, dom_gbs = gath_b, att_us, att_gbs
     traffic = traffic_lookup(dom, args.workload)
 
     # end to end through the host-buffer entry point
@@ -529,7 +538,9 @@ def run_ours(args):
         "gpu_launches": launches * args.steps,
         "kernels_per_step": launches,
         "graph_kernel_nodes_per_step": n_nodes,
-        "path": ("score -> top-k -> persistent attention (programmatic dependent launches; "
+        "path": ("one cooperative launch: score slices -> per-head top-k -> tensor-core "
+                 "attention" if plan == 3 else
+                 "score -> top-k -> persistent attention (programmatic dependent launches; "
                  + ("whole-block tensor-core kernel)" if plan == 2 else "CUDA-core kernel)")
                  if plan in (1, 2) else f"score -> top-k -> split-K attention (plan {plan})"),
         "cpu_baseline": cpu,
@@ -569,7 +580,7 @@ def _time_graph(g, stream, seconds, min_iters=5):
     return e0.elapsed_time(e1) / n, n
 
 
-def measure_decode_config(name, dev, seconds, pk, score_reduce="sum"):
+def measure_decode_config(name, dev, seconds, pk, score_reduce="sum", workload=None):
     """Decode-step throughput of one decode config (graph-replayed steps; L2
     defeated by rotating store replicas, or by an L2-sized write between
     steps whose own time is subtracted when replicas would not fit).
@@ -577,7 +588,7 @@ def measure_decode_config(name, dev, seconds, pk, score_reduce="sum"):
     import torch
     import retrieval_block_sparse_b200 as rba
     from retrieval_block_sparse_b200 import synth
-    w = synth.WORKLOADS[name]
+    w = workload if workload is not None else synth.WORKLOADS[name]
     x = synth.decode_inputs(w)
 
     def new_store():
@@ -586,8 +597,8 @@ def measure_decode_config(name, dev, seconds, pk, score_reduce="sum"):
                          dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep, device=dev,
                          score_reduce=score_reduce)
     st = new_store()
-    st.k.copy_(_to_dev(x["K"], w.dtype, dev))
-    st.v.copy_(_to_dev(x["V"], w.dtype, dev))
+    st.kv_rows(st.k).copy_(_to_dev(x["K"], w.dtype, dev))
+    st.kv_rows(st.v).copy_(_to_dev(x["V"], w.dtype, dev))
     aux = None
     if w.rep_mode == "topr_attn":
         aux = _to_dev(x["probe"], w.dtype, dev)
@@ -655,12 +666,13 @@ def measure_decode_config(name, dev, seconds, pk, score_reduce="sum"):
     us = ms * 1e3
     gbs = nbytes / (us * 1e-6) / 1e9
     plan = st.decode_plan(w.top_k, w.context, w.sink, w.window)
-    return {"workload": name, "score_reduce": score_reduce,
+    return {"workload": name, "head_dim": w.head_dim, "score_reduce": score_reduce,
             "steps_per_s": round(1e6 / us, 2), "us_per_step": round(us, 3),
             "algorithmic_bytes": nbytes, "rep_key_bytes": rep_b, "gathered_kv_bytes": gath_b,
             "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
             "path": {1: "pipelined, persistent attention (CUDA cores)",
-                     2: "pipelined, persistent attention (whole-block, tensor cores)"}.get(
+                     2: "pipelined, persistent attention (whole-block, tensor cores)",
+                     3: "one cooperative launch (score, top-k, tensor-core attention)"}.get(
                          plan, "split-K attention"),
             "steps_timed": n * len(stores),
             "l2": (f"L2-sized write between steps, its time subtracted" if use_flush else
@@ -668,21 +680,21 @@ def measure_decode_config(name, dev, seconds, pk, score_reduce="sum"):
                    f" >= 4 x L2)")}
 
 
-def measure_prefill_config(name, dev, seconds, pk):
+def measure_prefill_config(name, dev, seconds, pk, workload=None):
     """Chunked-prefill step of one prefill config: selection (score + top-k)
     and the retrieval-causal tensor-core attention, timed apart."""
     import torch
     import retrieval_block_sparse_b200 as rba
     from retrieval_block_sparse_b200 import synth
-    w = synth.WORKLOADS[name]
+    w = workload if workload is not None else synth.WORKLOADS[name]
     x = synth.prefill_inputs(w)
     mode = "embed_cosine" if w.score_mode == "cosine" else (
         "identity" if w.block_size == 1 else "mean")
     st = rba.Store(batch=1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
                    block_size=w.block_size, capacity_tokens=w.context, dtype=w.dtype, mode=mode,
                    d_ret=w.d_ret, device=dev)
-    st.k.copy_(_to_dev(x["K"], w.dtype, dev))
-    st.v.copy_(_to_dev(x["V"], w.dtype, dev))
+    st.kv_rows(st.k).copy_(_to_dev(x["K"], w.dtype, dev))
+    st.kv_rows(st.v).copy_(_to_dev(x["V"], w.dtype, dev))
     del x["K"], x["V"]
     nb = w.context // w.block_size
     if mode == "embed_cosine":
@@ -736,7 +748,8 @@ def measure_prefill_config(name, dev, seconds, pk):
         w.n_kv_heads * nc * w.head_dim * 2 if mode == "identity" else
         w.n_kv_heads * nc * w.head_dim * 4)
     del topk_ws
-    res = {"workload": name, "attend_us": round(ms_a * 1e3, 2), "attend_calls_timed": n_a,
+    res = {"workload": name, "head_dim": w.head_dim, "attend_us": round(ms_a * 1e3, 2),
+           "attend_calls_timed": n_a,
            "pairs": pairs, "flops": flops, "attend_tflops": round(tflops, 1),
            "attend_frac_of_bf16_peak": round(tflops / pk["bf16_tflops"], 4),
            "bf16_peak_tflops": pk["bf16_tflops"], "select_us": round(ms_s * 1e3, 2),
@@ -746,6 +759,103 @@ def measure_prefill_config(name, dev, seconds, pk):
         res["select_gbs"] = round(scan / (ms_s * 1e-3) / 1e9, 1)
         res["select_frac_of_hbm"] = round(scan / (ms_s * 1e-3) / 1e9 / pk["hbm_gbs"], 4)
     return res
+
+
+def measure_approx_config(dev, seconds, pk, group=64, kept=256):
+    """Two-stage approximate token retrieval (RetrievalAttention summary,
+    "proposed method") on the 1M-token decode shape with drift keys (nearby
+    keys resemble each other; the regime a group-mean index exploits): per
+    step rba_approx_select + rba_attend, graph-replayed with an L2-sized write
+    between steps whose own time is subtracted.  Reports recall of its tokens
+    against the exact top-k of the same store (rba_score + rba_topk), keys and
+    bytes read per step, and the exact step on the same store for contrast."""
+    import torch
+    import retrieval_block_sparse_b200 as rba
+    from retrieval_block_sparse_b200 import synth
+    w = synth.WORKLOADS["token-retrieval-decode-1m"].scaled(recipe="drift")
+    x = synth.decode_inputs(w)
+    st = rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                   head_dim=w.head_dim, block_size=1, capacity_tokens=w.context,
+                   dtype=w.dtype, mode="identity", device=dev)
+    st.k.copy_(_to_dev(x["K"], w.dtype, dev))
+    st.v.copy_(_to_dev(x["V"], w.dtype, dev))
+    del x["K"], x["V"]
+    q = _to_dev(x["q"], w.dtype, dev)
+    means = st.group_means(group)
+    BH = w.batch * w.n_kv_heads
+    idx = torch.empty((w.batch, w.n_kv_heads, w.top_k), dtype=torch.int32, device=dev)
+    groups = torch.empty((w.batch, w.n_kv_heads, kept), dtype=torch.int32, device=dev)
+    scanned = torch.empty((w.batch, w.n_kv_heads), dtype=torch.int32, device=dev)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.batch, w.n_q_heads), dtype=torch.float32, device=dev)
+    n = rba.lib().rba_approx_select_workspace_size(st.handle, w.context, w.sink, w.window,
+                                                   group, kept, w.top_k)
+    sel_ws = torch.zeros(max(n, 16), dtype=torch.uint8, device=dev)
+    att_ws = st.attend_workspace(w.top_k, w.context, w.sink, w.window)
+    step_ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)
+    eidx = torch.empty_like(idx)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(4 * l2, dtype=torch.uint8, device=dev)
+
+    def approx_step():
+        st.approx_select(q, w.context, w.sink, w.window, group, kept, w.top_k, means, idx=idx,
+                         groups_out=groups, scanned=scanned, workspace=sel_ws)
+        st.attend(q, idx, w.context, w.sink, w.window, out=out, lse=lse, workspace=att_ws)
+
+    def exact_step():
+        st.decode_step(q, w.top_k, w.context, w.sink, w.window, workspace=step_ws, idx=eidx,
+                       out=out, lse=lse)
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        approx_step()
+        exact_step()
+    torch.cuda.synchronize()
+    st.check()
+    a_idx, e_idx = idx.cpu().numpy(), eidx.cpu().numpy()
+    recall = float(np.mean([len(set(a_idx[b, h]) & set(e_idx[b, h])) / w.top_k
+                            for b in range(w.batch) for h in range(w.n_kv_heads)]))
+    graphs = {}
+    for name, fn in (("approx", approx_step), ("exact", exact_step), ("flush", None)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            flush.fill_(1)
+            if fn is not None:
+                fn()
+        graphs[name] = g
+    ms_f, _ = _time_graph(graphs["flush"], stream, seconds / 4)
+    ms_a, n_a = _time_graph(graphs["approx"], stream, seconds)
+    ms_e, _ = _time_graph(graphs["exact"], stream, seconds)
+    st.check()
+    us_a, us_e = (ms_a - ms_f) * 1e3, (ms_e - ms_f) * 1e3
+    keys_read = int(scanned.cpu().numpy().astype(np.int64).sum())
+    first, nc = st.candidates(w.context, w.sink, w.window)
+    n_groups = int(count_groups(w, group))
+    es = 2 if w.dtype == "bf16" else 4
+    att_tokens = w.top_k + min(w.sink, w.context - w.window) + w.window
+    bytes_a = BH * (n_groups * w.head_dim * 4 + kept * group * w.head_dim * es) + \
+        BH * att_tokens * w.head_dim * es * 2
+    bytes_e = BH * nc * w.head_dim * es + BH * att_tokens * w.head_dim * es * 2
+    return {"workload": "token-retrieval-decode-1m (drift keys)", "group": group,
+            "groups_kept": kept, "recall_vs_exact_top_k": round(recall, 4),
+            "keys_read_per_step": keys_read,
+            "keys_read_frac": round(keys_read / (BH * nc), 4),
+            "us_per_step": round(us_a, 2), "steps_per_s": round(1e6 / us_a, 1),
+            "algorithmic_bytes": bytes_a,
+            "achieved_gbs": round(bytes_a / (us_a * 1e-6) / 1e9, 1),
+            "frac_of_hbm": round(bytes_a / (us_a * 1e-6) / 1e9 / pk["hbm_gbs"], 4),
+            "exact_us_per_step": round(us_e, 2), "exact_algorithmic_bytes": bytes_e,
+            "speedup_vs_exact": round(us_e / us_a, 2), "steps_timed": n_a,
+            "l2": "L2-sized write between steps, its time subtracted",
+            "index": "group means (fp32) built once by rba_group_means, not timed"}
+
+
+def count_groups(w, group):
+    """Candidate groups of `group` tokens (full groups meeting [sink, T - window))."""
+    w0 = max(w.context - w.window, 0)
+    lo = w.sink // group
+    hi = min(-(-w0 // group), w.context // group)
+    return max(hi - lo, 0)
 
 
 def measure_memory_update(name, dev, trials, pk):
@@ -829,8 +939,17 @@ def measure_configs(dev, seconds):
         "infllm-decode-128k", dev, seconds, pk, score_reduce="max")
     for name in ("memlong-cosine-prefill", "token-retrieval-prefill-1m"):
         out[name] = measure_prefill_config(name, dev, seconds, pk)
+    # head dim 100 (MemLong's OpenLLaMA-3B: 32 heads of 100), pool rows padded to 128
+    from retrieval_block_sparse_b200 import synth
+    out["infllm-decode-128k:head-dim-100"] = measure_decode_config(
+        "infllm-decode-128k", dev, seconds, pk,
+        workload=synth.WORKLOADS["infllm-decode-128k"].scaled(head_dim=100))
+    out["memlong-cosine-prefill:head-dim-100"] = measure_prefill_config(
+        "memlong-cosine-prefill", dev, seconds, pk,
+        workload=synth.WORKLOADS["memlong-cosine-prefill"].scaled(head_dim=100))
     for name in ("memlong-cosine-prefill", "infllm-decode-128k"):
         out["memory-update:" + name] = measure_memory_update(name, dev, 10, pk)
+    out["token-retrieval-decode-1m:two-stage"] = measure_approx_config(dev, seconds, pk)
     return out
 
 
@@ -964,6 +1083,10 @@ def main(argv=None):
         torch.cuda.set_device(0)
         dev = torch.device("cuda", 0)
         from retrieval_block_sparse_b200 import synth
+        if args.only_config == "token-retrieval-decode-1m:two-stage":
+            print(json.dumps({"config": measure_approx_config(dev, args.config_seconds,
+                                                              peaks())}), flush=True)
+            return
         if args.only_config.startswith("memory-update:"):
             res = measure_memory_update(args.only_config.split(":", 1)[1], dev, 10, peaks())
             print(json.dumps({"config": res}), flush=True)

@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
   RBA_OK = 0,
   RBA_ERR_INVALID_ARG = 1,  /* bad size, pointer, mode or layout; nothing launched */
-  RBA_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. head_dim outside {64,128}) */
+  RBA_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. a head dim above 128) */
   RBA_ERR_WORKSPACE = 3,    /* workspace smaller than *_workspace_size() */
   RBA_ERR_CUDA = 4,         /* a CUDA runtime call failed */
   RBA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (status word) */
@@ -72,12 +72,12 @@ typedef enum { RBA_F32 = 0, RBA_BF16 = 1 } rba_dtype;
 
 /* How a block is represented for scoring ([ML] 2.3.2 memorisation). */
 typedef enum {
-  RBA_REP_MEAN = 0,         /* mean of the block's keys; rep pool fp32 [B][Hkv][cap_blocks][1][D] */
+  RBA_REP_MEAN = 0,         /* mean of the block's keys; rep pool fp32 [B][Hkv][cap_blocks][1][P] */
   RBA_REP_TOPR_ATTN = 1,    /* [IL] method: the n_rep keys that received the most attention from a
-                               probe; rep pool dtype [B][Hkv][cap_blocks][n_rep][D], positions
+                               probe; rep pool dtype [B][Hkv][cap_blocks][n_rep][P], positions
                                int32 [B][Hkv][cap_blocks][n_rep] */
   RBA_REP_EXTERNAL = 2,     /* [LM] landmark keys given by the caller; rep pool dtype
-                               [B][Hkv][cap_blocks][n_rep][D] */
+                               [B][Hkv][cap_blocks][n_rep][P] */
   RBA_REP_EMBED_COSINE = 3, /* [ML] 2.2.2: L2-normalised chunk embedding; rep pool fp32
                                [B][cap_blocks][d_ret]; scored by cosine */
   RBA_REP_IDENTITY = 4      /* [RA]: block size 1, each key is its own representation; no rep pool */
@@ -87,7 +87,7 @@ typedef struct {
   int32_t batch;            /* B */
   int32_t n_q_heads;        /* Hq (a multiple of n_kv_heads; q head i reads kv head i / (Hq/Hkv)) */
   int32_t n_kv_heads;       /* Hkv */
-  int32_t head_dim;         /* D: 64 or 128 */
+  int32_t head_dim;         /* D: a multiple of 4 up to 128; pool rows hold rba_row_pitch(D) */
   int32_t block_size;       /* bs >= 1 */
   int32_t n_rep;            /* r: representative keys per block (1 except RBA_REP_TOPR_ATTN / EXTERNAL) */
   int32_t d_ret;            /* embedding size (RBA_REP_EMBED_COSINE), else 0 */
@@ -107,7 +107,8 @@ typedef enum {
 typedef struct rba_store rba_store;
 
 /* Describe a block store ([ML] 2.2.2: memory = K-V pairs + representations).
- *   k_pool, v_pool  device, dtype [B][Hkv][capacity_tokens][D]
+ * P = rba_row_pitch(D) is the row length of every pool (P = D for D = 64 or 128).
+ *   k_pool, v_pool  device, dtype [B][Hkv][capacity_tokens][P]
  *   rep_pool        device, layout per mode above (NULL for RBA_REP_IDENTITY)
  *   rep_pos         device int32 [B][Hkv][cap_blocks][n_rep] for RBA_REP_TOPR_ATTN (may be
  *                   NULL: positions are then not recorded), else ignored
@@ -126,6 +127,16 @@ rba_status rba_store_destroy(rba_store* store);
  * represented by their most-attended tokens; this reading weighs the best one alone).
  * Errors: INVALID_ARG (unknown value; RBA_SCORE_MAX on cosine or identity stores). */
 rba_status rba_store_set_score_reduce(rba_store* store, int32_t reduce);
+
+/* Bound, in nanoseconds, of every device-side wait of the one-launch decode step on
+ * this store (host only; 0 restores the default of 2 s).  A wait that runs out
+ * records RBA_ERR_TIMEOUT in the status word; the kernel then stops issuing work,
+ * waits for its own copies in flight and returns, and every (batch, kv head) of the
+ * call still leaves its synchronisation words zero, so the next call on the same
+ * workspace runs normally.  Outputs of a call that timed out are undefined.  Meant
+ * for tests of that path and for callers that prefer a short bound.
+ * Errors: INVALID_ARG (NULL store). */
+rba_status rba_store_set_wait_limit_ns(rba_store* store, uint64_t ns);
 
 /* Candidate range for a store holding T tokens with the given sink/window
  * (host only; see the vocabulary above).  Errors: INVALID_ARG (tail block
@@ -230,6 +241,23 @@ rba_status rba_attend_noalloc(const rba_store* store, const void* q, const int32
                               int32_t k, int64_t T, int32_t sink, int32_t window, float scale,
                               float* out, float* lse, cudaStream_t stream);
 
+/* Landmark-gated decode attention ([LM] proposed method: a block's landmark token
+ * is the gate through which attention reaches the block).  The page gives no formula;
+ * the reading taken: the landmark takes the block's place in the query's softmax.
+ * For q head i of kv head h, with x_t = scale q . k_t:
+ *   out = (sum_{t local} e^{x_t} v_t + sum_j e^{y_j} o_j) / Z,   lse = ln Z,
+ *   local = sink U window tokens; j over the retrieved blocks idx[b][h][.];
+ *   y_j = scale q . L_j with L_j the block's landmark key (the rep pool);
+ *   o_j = sum over the block's tokens in [sink, w0) of softmax_block(x)_t v_t;
+ *   Z = sum_{t local} e^{x_t} + sum_j e^{y_j}.
+ * With every y_j equal to its block's log-sum-exp of x this is rba_attend.
+ * RBA_REP_EXTERNAL stores with n_rep = 1.  Arguments and layouts as rba_attend
+ * (no workspace).  Errors: INVALID_ARG, CUDA; out-of-range idx entries are skipped
+ * and flagged as RBA_ERR_BOUNDS in the status word. */
+rba_status rba_attend_landmark_gated(const rba_store* store, const void* q, const int32_t* idx,
+                                     int32_t k, int64_t T, int32_t sink, int32_t window,
+                                     float scale, float* out, float* lse, cudaStream_t stream);
+
 /* Chunked prefill, retrieval-causal ([ML] 2.3.3 / Figure 3): every row of a
  * query chunk attends bidirectionally to sink U retrieved blocks U window of
  * the memory, and causally to the chunk's own tokens (own token i' visible to
@@ -241,7 +269,9 @@ rba_status rba_attend_noalloc(const rba_store* store, const void* q, const int32
  *   out        device fp32 [n_chunks][Hq][chunk_len][D];  lse fp32 [n_chunks][Hq][chunk_len] or NULL
  *   The store's batch is 1 (one memory shared by all chunks) or n_chunks.
  *   workspace >= rba_attend_prefill_workspace_size().
- * Errors: INVALID_ARG, UNSUPPORTED (dtype other than bf16, D != 128), WORKSPACE, CUDA. */
+ *   Head dims between 64 and 128 run on 128-wide tiles: Q and the chunk's K/V are
+ *   copied, zero-padded, into the workspace (counted by the size call).
+ * Errors: INVALID_ARG, UNSUPPORTED (dtype other than bf16, D <= 64), WORKSPACE, CUDA. */
 rba_status rba_attend_prefill(const rba_store* store, const void* q, int32_t n_chunks,
                               int32_t chunk_len, const int32_t* idx, int32_t n_sel, int32_t k,
                               int64_t T, int32_t sink, int32_t window, const void* chunk_k,
@@ -252,15 +282,20 @@ size_t rba_attend_prefill_workspace_size(const rba_store* store, int32_t n_chunk
                                          int32_t sink, int32_t window);
 
 /* One whole decode step: rba_score (dot modes) -> rba_topk per (b, kv head)
- * -> rba_attend, with the same definitions as those calls, as three kernels
- * on `stream`.  Where rba_decode_step_plan() reports 1 or 2, the top-k kernel and
- * the persistent attention kernel are programmatic dependents of the kernel
- * before them: they start early, the attention kernel streams the sink and
- * window rows, and each waits on the device for its inputs.
+ * -> rba_attend, with the same definitions as those calls, on `stream`.
+ * Where rba_decode_step_plan() reports 3 it is ONE cooperative launch of one CTA
+ * per SM: the CTAs of a (batch, kv head) score slices of its candidates, each
+ * selects the head's top k once all slices are published, and they stream the
+ * sink/window rows meanwhile and the selected rows after.  Where it reports 1 or
+ * 2 it is three kernels, the top-k kernel and the persistent attention kernel
+ * programmatic dependents of the kernel before them; else three kernels in
+ * stream order.
  *   q device dtype [B][Hq][D]; idx device int32 [B][Hkv][k] (written); scores device fp32
  *   [B][Hkv][nc] (written) or NULL; out/lse as rba_attend.
- *   workspace >= rba_decode_step_workspace_size(); it starts with rba_attend's workspace,
- *   whose ticket words must be zero before the first call.
+ *   workspace >= rba_decode_step_workspace_size(); zero it before the first call (its
+ *   synchronisation words must start at zero; every call that completes leaves them
+ *   zero, and their offsets depend on the store only, so one workspace of the largest
+ *   size serves calls of every geometry).
  * Errors: as the three calls. */
 rba_status rba_decode_step(const rba_store* store, const void* q, int32_t k, int64_t T,
                            int32_t sink, int32_t window, float scale, float* scores,
@@ -270,6 +305,11 @@ size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t
                                       int32_t sink, int32_t window);
 
 /* How rba_decode_step runs this problem (host only; queries the device, launches nothing):
+ *   3   the whole step in one cooperative launch: bf16 store, block size a multiple of 64,
+ *       head dim 64 or 128, GQA group of 1, 2 or 4, dot-mode representations (mean, top-r,
+ *       landmark) with at most 8 keys per block, 1 <= k <= 256, at most 4096 candidates
+ *       per (batch, kv head), at most half as many (batch, kv head) units as SMs, and a
+ *       part's slice of representative keys within 64 KiB
  *   2   score -> top-k -> persistent attention kernel, the last two as programmatic
  *       dependents (overlapped); the attention kernel is the whole-block one: bf16 store,
  *       block size a multiple of 64, head dim 64 or 128; inner products on tensor cores
@@ -283,9 +323,9 @@ int32_t rba_decode_step_plan(const rba_store* store, int32_t k, int64_t T, int32
                              int32_t window);
 
 /* Number of kernels rba_decode_step enqueues for this problem (host only, launches
- * nothing): block scores and top-k (one kernel for rows of up to 8192 candidates, four
- * above; neither when k = 0), then one attention kernel (persistent or split-K).  -4 for
- * invalid arguments. */
+ * nothing): 1 where rba_decode_step_plan() reports 3; else block scores and top-k (one
+ * kernel for rows of up to 8192 candidates, four above; neither when k = 0), then one
+ * attention kernel (persistent or split-K).  -4 for invalid arguments. */
 int32_t rba_decode_step_launches(const rba_store* store, int32_t k, int64_t T, int32_t sink,
                                  int32_t window);
 
@@ -310,6 +350,45 @@ rba_status rba_stream_step(rba_store* store, const void* q, const void* k_new,
                            float scale, const void* aux, int32_t n_aux, int32_t* idx, float* out,
                            float* lse, int32_t* k_used, void* workspace, size_t ws_bytes,
                            cudaStream_t stream);
+
+/* Two-stage approximate token retrieval for block size 1 ([RA] proposed method:
+ * the few keys that matter are found by an approximate search that reads 1-3 % of
+ * the keys instead of all of them).  The page names no index; this one is the
+ * plainest the rest supports: consecutive groups of `group` tokens represented by
+ * the mean of their keys.
+ *
+ * rba_group_means: the index.  For groups j in [first_group, first_group + n_groups)
+ * of every (batch, kv head), means[b][h][j] = (1 / group) sum_t K[j * group + t]
+ * (fp32).  RBA_REP_IDENTITY stores only.
+ *   means  device fp32 [B][Hkv][capacity_tokens / group][P], caller-owned
+ * Errors: INVALID_ARG (not an identity store, groups beyond the capacity), CUDA. */
+rba_status rba_group_means(const rba_store* store, int64_t first_group, int32_t n_groups,
+                           int32_t group, float* means, cudaStream_t stream);
+
+/* rba_approx_select: per (batch, kv head), with the GQA group's queries summed
+ *   stage 1  every candidate group (a full group meeting [sink, T - window)) scored
+ *            by its mean; the best `groups_kept` kept (ties -> lower group);
+ *   stage 2  every token of the kept groups that lies in [sink, T - window) scored
+ *            exactly (q . k_t); the best k kept (ties -> lower token).
+ * The keys read are one mean per candidate group plus the kept groups' tokens.
+ * Attend over the result with rba_attend (block size 1: token ids are block ids).
+ *   q           device dtype [B][Hq][D]
+ *   means       device fp32 index from rba_group_means, covering the candidate groups
+ *   idx         device int32 [B][Hkv][k], written: the selected tokens, ascending
+ *   groups_out  device int32 [B][Hkv][groups_kept] (kept groups, ascending) or NULL
+ *   scanned     device int32 [B][Hkv] (keys read) or NULL
+ *   workspace >= rba_approx_select_workspace_size()
+ * Requires groups_kept * group >= k + 2 * group (enough candidate tokens in any
+ * kept set) and groups_kept <= the candidate groups.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+rba_status rba_approx_select(const rba_store* store, const void* q, int64_t T, int32_t sink,
+                             int32_t window, int32_t group, int32_t groups_kept, int32_t k,
+                             const float* means, int32_t* idx, int32_t* groups_out,
+                             int32_t* scanned, void* workspace, size_t ws_bytes,
+                             cudaStream_t stream);
+size_t rba_approx_select_workspace_size(const rba_store* store, int64_t T, int32_t sink,
+                                        int32_t window, int32_t group, int32_t groups_kept,
+                                        int32_t k);
 
 /* Dynamic memory update ([ML] 2.3.2, dynamic memory update): retrieval
  * counters decide what the memory keeps once it overflows.  The newest entries
@@ -381,6 +460,15 @@ rba_status rba_decode_step_host(const rba_store* store, const void* q_host, void
 /* Synchronises `stream`, reads the store's status word, clears it, and returns
  * the first device-side error recorded since the last check (RBA_OK if none). */
 rba_status rba_store_check(const rba_store* store, cudaStream_t stream);
+
+/* Row pitch (elements) of the K/V and representation pools for a head dim D
+ * (host only): 64 for D <= 64, else 128; -1 for an unsupported D (not a multiple
+ * of 4, or above 128).  Pools hold each row in `pitch` elements: the first D are
+ * the row, the rest are padding that must hold zeros (the library's own writes
+ * -- rba_memorize, rba_stream_step, rba_memory_update -- keep them zero).  Every
+ * other tensor of the interface (q, out, K/V and key inputs, prefill chunks) is
+ * dense with rows of D elements. */
+int32_t rba_row_pitch(int32_t head_dim);
 
 const char* rba_status_string(rba_status status);
 int32_t rba_version(void);

@@ -41,7 +41,10 @@ def two_stage_select(qs, K, T: int, *, group: int, sink: int, window: int, group
 
     qs [m][D] the queries sharing the selection; K [>= T][D] the keys (fp64).
     Returns dict: tokens (k, ascending), groups (kept group ids, ascending),
-    scanned (keys read: one mean per candidate group + the kept groups' tokens)."""
+    scanned (keys read: one mean per candidate group + the kept groups' tokens),
+    and the two stages' inputs: cand_groups (candidate group ids), group_scores
+    (their stage-1 scores), kept_tokens (the kept groups' candidate tokens,
+    ascending) and token_scores (their stage-2 scores)."""
     K = np.asarray(K, dtype=np.float64)
     w0 = max(T - window, 0)
     groups = candidate_blocks(T, group, sink, window)
@@ -55,7 +58,8 @@ def two_stage_select(qs, K, T: int, *, group: int, sink: int, window: int, group
         raise ValueError("the kept groups hold fewer than k candidate tokens")
     s2 = score_dot(qs, K[toks][:, None, :])
     return {"tokens": toks[top_k(s2, k)], "groups": kept,
-            "scanned": int(groups.size + toks.size)}
+            "scanned": int(groups.size + toks.size),
+            "cand_groups": groups, "group_scores": s1, "kept_tokens": toks, "token_scores": s2}
 
 
 def recall(approx_tokens, exact_tokens) -> float:

@@ -8,6 +8,7 @@
 // partials by log-sum-exp (no CTA ever waits for another).
 #include "attend_impl.cuh"
 #include "decode_fused.cuh"
+#include "decode_step.cuh"
 #include "score_impl.cuh"
 #include "topk_impl.cuh"
 
@@ -117,7 +118,7 @@ size_t attend_workspace_bytes(int BH, int Hq_total, int D, int nsplit) {
 size_t splitk_workspace_bytes(const rba_store* st, const Geometry& g, int k) {
   const int BH = st->d.batch * st->d.n_kv_heads;
   const int nsplit = attend_nsplit(BH, n_att_bound(g, k));
-  return attend_workspace_bytes(BH, st->d.batch * st->d.n_q_heads, st->d.head_dim, nsplit);
+  return attend_workspace_bytes(BH, st->d.batch * st->d.n_q_heads, st->pitch, nsplit);
 }
 
 rba_status launch_attend(const rba_store* st, const void* q, const int32_t* idx, int k,
@@ -127,7 +128,7 @@ rba_status launch_attend(const rba_store* st, const void* q, const int32_t* idx,
   const int BH = d.batch * d.n_kv_heads;
   const int G = d.n_q_heads / d.n_kv_heads;
   const int nsplit = attend_nsplit(BH, n_att_bound(g, k));
-  AttendWs w = attend_layout(ws, BH, d.batch * d.n_q_heads, d.head_dim, nsplit);
+  AttendWs w = attend_layout(ws, BH, d.batch * d.n_q_heads, st->pitch, nsplit);
   if (ws == nullptr || ws_bytes < w.bytes) return RBA_ERR_WORKSPACE;
   AttendArgs a;
   a.K = st->k;
@@ -151,12 +152,13 @@ rba_status launch_attend(const rba_store* st, const void* q, const int32_t* idx,
   a.nsplit = nsplit;
   a.first = g.first;
   a.nc = g.nc;
+  a.qd = d.head_dim;
   a.scale_log2 = scale * 1.4426950408889634f;
   if (d.dtype == RBA_BF16) {
-    if (d.head_dim == 128) return dispatch_g<__nv_bfloat16, 128>(a, G, BH, stream);
+    if (st->pitch == 128) return dispatch_g<__nv_bfloat16, 128>(a, G, BH, stream);
     return dispatch_g<__nv_bfloat16, 64>(a, G, BH, stream);
   }
-  if (d.head_dim == 128) return dispatch_g<float, 128>(a, G, BH, stream);
+  if (st->pitch == 128) return dispatch_g<float, 128>(a, G, BH, stream);
   return dispatch_g<float, 64>(a, G, BH, stream);
 }
 
@@ -182,7 +184,7 @@ AttendLayout attend_layout_full(void* ws, const rba_store* st, const Geometry& g
   l.fused_sync = p + off;
   off += fused_sync_bytes(st);
   const int nsplit = attend_nsplit(BH, n_att_bound(g, k));
-  l.splitk_bytes = attend_workspace_bytes(BH, d.batch * d.n_q_heads, d.head_dim, nsplit);
+  l.splitk_bytes = attend_workspace_bytes(BH, d.batch * d.n_q_heads, st->pitch, nsplit);
   l.splitk_ws = p + off;
   off += align_up(l.splitk_bytes, 256);
   l.fused_slots = reinterpret_cast<float*>(p + off);
@@ -210,19 +212,34 @@ rba_status attend_any(const rba_store* st, const void* q, const int32_t* idx, in
 
 struct StepWs {
   AttendLayout att;
+  bool one_launch;      // the one-launch decode step covers the problem
+  void* step_sync;      // its synchronisation words (zero between calls)
+  float* step_slots;    // its partial-state slots
   float* scores;
   void* topk_ws;
   size_t topk_bytes;
   size_t total;
 };
 
-// [attention workspace] [scores] [top-k scratch]
+// [one-launch step: sync words] [attention workspace] [one-launch step: slots]
+// [scores] [top-k scratch].  The zero words (the step's, then the attention
+// kernels' at the start of the attention workspace) sit at offsets that
+// depend on the store alone, so calls of any geometry on one workspace agree
+// on them.
 StepWs step_layout(void* ws, const rba_store* st, const Geometry& g, int k, bool own_scores) {
   const int BH = st->d.batch * st->d.n_kv_heads;
   StepWs s;
   char* p = static_cast<char*>(ws);
-  s.att = attend_layout_full(ws, st, g, k);
-  size_t off = align_up(s.att.total, 256);
+  s.step_sync = p;
+  size_t off = step_sync_bytes(st);
+  s.att = attend_layout_full(p + off, st, g, k);
+  off += align_up(s.att.total, 256);
+  s.one_launch = step_eligible(st, g, k);
+  s.step_slots = nullptr;
+  if (s.one_launch) {
+    s.step_slots = reinterpret_cast<float*>(p + off);
+    off += step_slot_bytes(st);
+  }
   s.scores = nullptr;
   if (own_scores) {
     s.scores = reinterpret_cast<float*>(p + off);
@@ -281,6 +298,8 @@ rba_status rba_decode_step(const rba_store* st, const void* q, int32_t k, int64_
   const int BH = st->d.batch * st->d.n_kv_heads;
   const int grp = st->d.n_q_heads / st->d.n_kv_heads;
   if (grp > 64) return RBA_ERR_UNSUPPORTED;
+  if (w.one_launch)  // the whole step in one cooperative launch
+    return launch_step(st, q, k, g, scale, sc, idx, out, lse, w.step_sync, w.step_slots, stream);
   // score -> top-k -> attention; the top-k kernel and the persistent
   // attention kernel start early (programmatic dependent launch) and wait
   // for their inputs on the device
@@ -312,11 +331,14 @@ rba_status rba_stream_step(rba_store* st, const void* q, const void* k_new, cons
   const int32_t ke = k < g.nc ? k : g.nc;  // early in a stream fewer blocks are candidates
   if (k_used != nullptr) *k_used = ke;
   // 1. the new token's K and V at position T of every (batch, kv head)
+  // (the new rows are head_dim long; pool rows are st->pitch long, their
+  // padding columns stay zero)
   const size_t row = size_t(d.head_dim) * dtype_size(d.dtype);
+  const size_t prow = size_t(st->pitch) * dtype_size(d.dtype);
   const size_t rows = size_t(d.batch) * d.n_kv_heads;
-  const size_t pitch = size_t(d.capacity_tokens) * row;
-  char* kdst = static_cast<char*>(st->k) + size_t(T) * row;
-  char* vdst = static_cast<char*>(st->v) + size_t(T) * row;
+  const size_t pitch = size_t(d.capacity_tokens) * prow;
+  char* kdst = static_cast<char*>(st->k) + size_t(T) * prow;
+  char* vdst = static_cast<char*>(st->v) + size_t(T) * prow;
   RBA_CUDA_TRY(cudaMemcpy2DAsync(kdst, pitch, k_new, row, row, rows, cudaMemcpyDeviceToDevice,
                                  stream));
   RBA_CUDA_TRY(cudaMemcpy2DAsync(vdst, pitch, v_new, row, row, rows, cudaMemcpyDeviceToDevice,
@@ -338,6 +360,7 @@ int32_t rba_decode_step_plan(const rba_store* st, int32_t k, int64_t T, int32_t 
   Geometry g;
   if (st == nullptr || k < 0 || geometry(st, T, sink, window, &g) != RBA_OK || k > g.nc)
     return -4;
+  if (step_eligible(st, g, k)) return 3;
   if (!fused_eligible(st, g, k)) return 0;
   const int occ = fused_occupancy(st);
   if (occ < 0) return -3;
@@ -351,6 +374,7 @@ int32_t rba_decode_step_launches(const rba_store* st, int32_t k, int64_t T, int3
   Geometry g;
   if (st == nullptr || k < 0 || geometry(st, T, sink, window, &g) != RBA_OK || k > g.nc)
     return -4;
+  if (step_eligible(st, g, k)) return 1;  // the whole step in one launch
   int32_t n = 0;
   if (k > 0) n += 1 + (g.nc <= kSmallN ? 1 : 4);  // scores; top-k (one kernel, or four)
   return n + 1;  // the attention kernel (persistent or split-K)

@@ -28,6 +28,8 @@ struct AttendArgs {
   int64_t T;
   int64_t w0;
   int Hq, Hkv, k, bs, sink, sink_end, nsplit, first, nc;
+  int qd;                 // head dim: row length of q and out (the pools' rows hold D >= qd
+                          // elements, the columns past qd zero)
   float scale_log2;       // scale * log2(e)
 };
 
@@ -190,15 +192,18 @@ __device__ __forceinline__ void load_q(const AttendArgs& a, int bh, LaneState<T,
   const T* q = static_cast<const T*>(a.q);
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const T* qr = q + (int64_t(b) * a.Hq + h * grp + g0 + g) * D + part * C::EPL;
+    // q rows are qd long; columns past qd count as zero
+    const T* qr = q + (int64_t(b) * a.Hq + h * grp + g0 + g) * a.qd;
 #pragma unroll
     for (int j = 0; j < C::CPL; ++j) {
       const int jj = (j + rot) % C::CPL;
 #pragma unroll
       for (int e = 0; e < C::EPC; e += 2) {
+        const int col = part * C::EPL + jj * C::EPC + e;  // qd is even: col, col + 1 agree
         st.q[g][(j * C::EPC + e) / 2] =
-            make_float2(Elem<T>::to_f32(qr[jj * C::EPC + e]) * a.scale_log2,
-                        Elem<T>::to_f32(qr[jj * C::EPC + e + 1]) * a.scale_log2);
+            col < a.qd ? make_float2(Elem<T>::to_f32(qr[col]) * a.scale_log2,
+                                     Elem<T>::to_f32(qr[col + 1]) * a.scale_log2)
+                       : make_float2(0.f, 0.f);
       }
     }
     st.m[g] = -INFINITY;
@@ -408,13 +413,13 @@ __device__ __forceinline__ void merge_partials_last(const AttendArgs& a, int bh,
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int g = i / D, d = i % D;
+  for (int i = threadIdx.x; i < G * a.qd; i += blockDim.x) {
+    const int g = i / a.qd, d = i % a.qd;
     const float* p = a.part + (int64_t(bh) * G + g) * ns * (D + 2) + 2 + d;
     float acc = 0.f;
     for (int s = 0; s < ns; ++s) acc += wsm[g * ns + s] * __ldcg(p + s * (D + 2));
     const int b = bh / a.Hkv, h = bh % a.Hkv;
-    a.out[(int64_t(b) * a.Hq + h * G + g) * D + d] = acc;
+    a.out[(int64_t(b) * a.Hq + h * G + g) * a.qd + d] = acc;
   }
   if (threadIdx.x == 0) a.tickets[bh] = 0;
 }

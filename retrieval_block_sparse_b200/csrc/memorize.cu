@@ -25,6 +25,25 @@ __global__ void copy_rows_kernel(const uint4* __restrict__ src, uint4* __restric
   }
 }
 
+// As copy_rows_kernel for rows of src_words 32-bit words into rows of
+// dst_words >= src_words (head dims below the pools' row pitch): the words
+// past src_words are written as zero.
+__global__ void copy_rows_pad_kernel(const uint32_t* __restrict__ src, uint32_t* __restrict__ dst,
+                                     int64_t bh, int64_t rows, int64_t dst_rows, int64_t row0,
+                                     int32_t src_words, int32_t dst_words) {
+  const int64_t per_bh = rows * dst_words;
+  const int64_t total = bh * per_bh;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t s = i / per_bh;
+    const int64_t rem = i - s * per_bh;
+    const int64_t r = rem / dst_words;
+    const int w = static_cast<int>(rem - r * dst_words);
+    dst[(s * dst_rows + row0 + r) * dst_words + w] =
+        w < src_words ? src[(s * rows + r) * src_words + w] : 0u;
+  }
+}
+
 // RBA_REP_MEAN: rep[j] = (1/bs) sum_t k_t, fp32.  grid (n_blocks, B*Hkv), block D.
 template <typename T>
 __global__ void rep_mean_kernel(const T* __restrict__ K, float* __restrict__ rep, int D, int bs,
@@ -45,8 +64,8 @@ constexpr int kMaxProbe = 32;
 template <typename T, int D>
 __global__ void rep_topr_kernel(const T* __restrict__ K, const T* __restrict__ probe,
                                 T* __restrict__ rep, int32_t* __restrict__ rep_pos, int Hkv,
-                                int bs, int r, int P, float scale_log2, int64_t cap_tokens,
-                                int64_t cap_blocks, int64_t first_block) {
+                                int bs, int r, int P, int qd, float scale_log2,
+                                int64_t cap_tokens, int64_t cap_blocks, int64_t first_block) {
   extern __shared__ float sm[];
   float* sprobe = sm;                          // [P][D]
   float* sred = sm + P * D;                    // [32 warps][kMaxProbe]
@@ -57,8 +76,10 @@ __global__ void rep_topr_kernel(const T* __restrict__ K, const T* __restrict__ p
   const int64_t j = first_block + blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int h = static_cast<int>(bh % Hkv);
-  for (int i = t; i < P * D; i += blockDim.x)
-    sprobe[i] = Elem<T>::to_f32(probe[int64_t(h) * P * D + i]);
+  for (int i = t; i < P * D; i += blockDim.x) {  // probe rows are qd long
+    const int p = i / D, d = i - p * D;
+    sprobe[i] = d < qd ? Elem<T>::to_f32(probe[(int64_t(h) * P + p) * qd + d]) : 0.f;
+  }
   __syncthreads();
 
   const bool valid = t < bs;
@@ -200,21 +221,35 @@ extern "C" rba_status rba_memorize(rba_store* st, const void* k_src, const void*
   if ((k_src == nullptr) != (v_src == nullptr)) return RBA_ERR_INVALID_ARG;
   const int64_t BH = int64_t(d.batch) * d.n_kv_heads;
   const int64_t bs = d.block_size;
-  const int D = d.head_dim;
+  const int D = st->pitch;  // pool rows; inputs are d.head_dim long
   const size_t es = dtype_size(d.dtype);
   const int vec_row = static_cast<int>(D * es / 16);
+  const bool padded = d.head_dim != D;
+  const int src_words = static_cast<int>(d.head_dim * es / 4), dst_words = static_cast<int>(D * es / 4);
+  // rows of `rows` per (b, kv head) from a dense input into a pool at row0
+  auto copy_in = [&](const void* src, void* dst, int64_t rows, int64_t dst_rows,
+                     int64_t row0) -> rba_status {
+    if (!padded) {
+      const int g = grid_for(BH * rows * vec_row, 256);
+      copy_rows_kernel<<<g, 256, 0, stream>>>(static_cast<const uint4*>(src),
+                                              static_cast<uint4*>(dst), BH, rows, dst_rows, row0,
+                                              vec_row);
+    } else {
+      const int g = grid_for(BH * rows * dst_words, 256);
+      copy_rows_pad_kernel<<<g, 256, 0, stream>>>(static_cast<const uint32_t*>(src),
+                                                  static_cast<uint32_t*>(dst), BH, rows, dst_rows,
+                                                  row0, src_words, dst_words);
+    }
+    RBA_LAUNCH_CHECK();
+    return RBA_OK;
+  };
 
   if (k_src != nullptr) {
     const int64_t rows = int64_t(n_blocks) * bs;
-    const int g = grid_for(BH * rows * vec_row, 256);
-    copy_rows_kernel<<<g, 256, 0, stream>>>(static_cast<const uint4*>(k_src),
-                                            static_cast<uint4*>(st->k), BH, rows,
-                                            d.capacity_tokens, first_block * bs, vec_row);
-    RBA_LAUNCH_CHECK();
-    copy_rows_kernel<<<g, 256, 0, stream>>>(static_cast<const uint4*>(v_src),
-                                            static_cast<uint4*>(st->v), BH, rows,
-                                            d.capacity_tokens, first_block * bs, vec_row);
-    RBA_LAUNCH_CHECK();
+    rba_status s = copy_in(k_src, st->k, rows, d.capacity_tokens, first_block * bs);
+    if (s != RBA_OK) return s;
+    s = copy_in(v_src, st->v, rows, d.capacity_tokens, first_block * bs);
+    if (s != RBA_OK) return s;
   }
 
   const dim3 grid(static_cast<unsigned>(n_blocks), static_cast<unsigned>(BH));
@@ -243,8 +278,8 @@ extern "C" rba_status rba_memorize(rba_store* st, const void* k_src, const void*
     kfn<<<grid, threads, smem, stream>>>(static_cast<const T_*>(st->k),                       \
                                          static_cast<const T_*>(aux), static_cast<T_*>(st->rep), \
                                          st->rep_pos, d.n_kv_heads, static_cast<int>(bs),     \
-                                         d.n_rep, n_aux, sl2, d.capacity_tokens, st->cap_blocks, \
-                                         first_block);                                        \
+                                         d.n_rep, n_aux, d.head_dim, sl2, d.capacity_tokens,  \
+                                         st->cap_blocks, first_block);                        \
   } while (0)
       if (d.dtype == RBA_BF16) {
         if (D == 128) RBA_TOPR(__nv_bfloat16, 128); else RBA_TOPR(__nv_bfloat16, 64);
@@ -258,12 +293,9 @@ extern "C" rba_status rba_memorize(rba_store* st, const void* k_src, const void*
     case RBA_REP_EXTERNAL: {
       if (aux == nullptr) return RBA_ERR_INVALID_ARG;
       const int64_t rows = int64_t(n_blocks) * d.n_rep;
-      const int g = grid_for(BH * rows * vec_row, 256);
-      copy_rows_kernel<<<g, 256, 0, stream>>>(static_cast<const uint4*>(aux),
-                                              static_cast<uint4*>(st->rep), BH, rows,
-                                              st->cap_blocks * d.n_rep, first_block * d.n_rep,
-                                              vec_row);
-      RBA_LAUNCH_CHECK();
+      const rba_status s =
+          copy_in(aux, st->rep, rows, st->cap_blocks * d.n_rep, first_block * d.n_rep);
+      if (s != RBA_OK) return s;
       break;
     }
     case RBA_REP_EMBED_COSINE: {

@@ -311,15 +311,15 @@ extern "C" rba_status rba_memory_update(rba_store* st, int64_t T, int32_t pinned
   a.v = static_cast<uint4*>(st->v);
   a.cap_tokens = d.capacity_tokens;
   a.bs = static_cast<int32_t>(bs);
-  a.row_vecs = static_cast<int32_t>(d.head_dim * dtype_size(d.dtype) / 16);
+  a.row_vecs = static_cast<int32_t>(st->pitch * dtype_size(d.dtype) / 16);
   a.heads = d.mode == RBA_REP_EMBED_COSINE ? d.n_kv_heads : 1;
   a.units = units;
   a.rep = static_cast<uint32_t*>(st->rep);
   switch (d.mode) {
-    case RBA_REP_MEAN: a.rep_words = d.head_dim; break;
+    case RBA_REP_MEAN: a.rep_words = st->pitch; break;
     case RBA_REP_TOPR_ATTN:
     case RBA_REP_EXTERNAL:
-      a.rep_words = static_cast<int32_t>(d.n_rep * d.head_dim * dtype_size(d.dtype) / 4);
+      a.rep_words = static_cast<int32_t>(d.n_rep * st->pitch * dtype_size(d.dtype) / 4);
       break;
     case RBA_REP_EMBED_COSINE: a.rep_words = d.d_ret; break;
     default: a.rep_words = 0;

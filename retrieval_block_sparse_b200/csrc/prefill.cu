@@ -53,6 +53,7 @@ struct PrefillArgs {
   int staged;          // past tokens come from the staging buffer
   int n_att_max;       // staging rows per (chunk, kv head)
   int pairs_outer;     // grid order: 1 = (head, chunk, pair), heaviest pairs first
+  int od;              // row length of out (the head dim; tiles are kHD wide, zero-padded)
   float scale_log2;
 };
 
@@ -224,6 +225,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
 // The registers of an in-flight tcgen05.ld pass through this empty asm after
 // tcgen05.wait::ld, so the compiler cannot move their uses above the wait.
 __device__ __forceinline__ void tmem_regs_ready(float* v) {
@@ -598,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __all_sync(0xffffffffu, mbar_wait(&bars->o_done[X], (n_s - 1) & 1, bars, a.status, 9))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* orow = a.out + ((int64_t(c) * a.Hq + hq) * a.Nq + qpos) * kHD;
+      float* orow = a.out + ((int64_t(c) * a.Hq + hq) * a.Nq + qpos) * a.od;
 #pragma unroll 1
       for (int q4 = 0; q4 < 4; ++q4) {
         float o[32];
@@ -607,9 +609,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_regs_ready(o);
         if (qpos < a.Nq) {
 #pragma unroll
-          for (int x = 0; x < 32; x += 4)
-            *reinterpret_cast<float4*>(orow + q4 * 32 + x) =
-                make_float4(o[x] * inv, o[x + 1] * inv, o[x + 2] * inv, o[x + 3] * inv);
+          for (int x = 0; x < 32; x += 4)  // (od is a multiple of 4: whole float4s)
+            if (q4 * 32 + x < a.od)
+              *reinterpret_cast<float4*>(orow + q4 * 32 + x) =
+                  make_float4(o[x] * inv, o[x + 1] * inv, o[x + 2] * inv, o[x + 3] * inv);
         }
       }
       if (qpos < a.Nq && a.lse != nullptr)
@@ -687,6 +690,19 @@ __global__ void gather_kernel(PrefillArgs a, const __nv_bfloat16* __restrict__ K
   }
 }
 
+// rows of D bf16 (dense) -> rows of kHD with zero padding, in 32-bit words
+__global__ void pad_rows_kernel(const uint32_t* __restrict__ src, uint32_t* __restrict__ dst,
+                                int64_t rows, int src_words) {
+  constexpr int kDstWords = kHD / 2;
+  const int64_t total = rows * kDstWords;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / kDstWords;
+    const int w = static_cast<int>(i - r * kDstWords);
+    dst[i] = w < src_words ? src[r * src_words + w] : 0u;
+  }
+}
+
 // [rows][128] bf16 matrix, 128-byte-swizzled boxes of 64 columns x 128 rows
 bool make_map(CUtensorMap* m, const void* base, int64_t rows) {
   return make_tmap_bf16(m, base, rows, kHD, 128);
@@ -695,10 +711,13 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows) {
 struct Plan {
   bool staged;
   int n_att_max;
+  size_t staged_bytes;  // staging buffers of the gathered past K and V
+  bool padded;          // head dim below kHD: Q and the chunk's K/V padded to kHD columns
+  size_t q_pad, kv_pad; // bytes of the padded Q and of each padded chunk K / V
   size_t ws_bytes;
 };
 
-Plan plan(const rba_store* st, const Geometry& g, int n_chunks, int k) {
+Plan plan(const rba_store* st, const Geometry& g, int n_chunks, int chunk_len, int k) {
   Plan p;
   const rba_store_desc& d = st->d;
   const int64_t n_att = int64_t(g.sink_end) + (g.T - g.w0) + int64_t(k) * d.block_size;
@@ -707,7 +726,12 @@ Plan plan(const rba_store* st, const Geometry& g, int n_chunks, int k) {
                                (g.T - g.w0 + kBN - 1) / kBN;
   p.staged = d.block_size < kBN || direct_tiles > kMaxTiles / 2;
   p.n_att_max = static_cast<int>(n_att);
-  p.ws_bytes = p.staged ? align_up(size_t(n_chunks) * d.n_kv_heads * n_att * kHD * 2, 256) * 2 : 0;
+  p.staged_bytes =
+      p.staged ? align_up(size_t(n_chunks) * d.n_kv_heads * n_att * kHD * 2, 256) * 2 : 0;
+  p.padded = d.head_dim != kHD;
+  p.q_pad = p.padded ? align_up(size_t(n_chunks) * d.n_q_heads * chunk_len * kHD * 2, 256) : 0;
+  p.kv_pad = p.padded ? align_up(size_t(n_chunks) * d.n_kv_heads * chunk_len * kHD * 2, 256) : 0;
+  p.ws_bytes = p.staged_bytes + p.q_pad + 2 * p.kv_pad;
   return p;
 }
 
@@ -726,7 +750,9 @@ rba_status rba_attend_prefill(const rba_store* st, const void* q, int32_t n_chun
       chunk_v == nullptr || n_chunks <= 0 || chunk_len <= 0 || k < 0)
     return RBA_ERR_INVALID_ARG;
   const rba_store_desc& d = st->d;
-  if (d.dtype != RBA_BF16 || d.head_dim != kHD) return RBA_ERR_UNSUPPORTED;
+  // head dims below kHD run on kHD-wide tiles: pools are held with rows of kHD
+  // elements (zero padding), Q and the chunk's K/V are padded into the workspace
+  if (d.dtype != RBA_BF16 || st->pitch != kHD) return RBA_ERR_UNSUPPORTED;
   if (d.batch != 1 && d.batch != n_chunks) return RBA_ERR_INVALID_ARG;
   if (n_sel != 1 && n_sel != d.n_kv_heads) return RBA_ERR_INVALID_ARG;
   if (k > 0 && idx == nullptr) return RBA_ERR_INVALID_ARG;
@@ -734,7 +760,7 @@ rba_status rba_attend_prefill(const rba_store* st, const void* q, int32_t n_chun
   rba_status s = geometry(st, T, sink, window, &g);
   if (s != RBA_OK) return s;
   if (k > g.nc) return RBA_ERR_INVALID_ARG;
-  const Plan p = plan(st, g, n_chunks, k);
+  const Plan p = plan(st, g, n_chunks, chunk_len, k);
   const int64_t own_tiles = (chunk_len + kBN - 1) / kBN;
   if ((int64_t(p.n_att_max) + kBN - 1) / kBN + own_tiles > kMaxTiles) return RBA_ERR_UNSUPPORTED;
   if (int64_t(n_chunks) * d.n_q_heads * chunk_len >= (int64_t(1) << 31) ||
@@ -765,13 +791,14 @@ rba_status rba_attend_prefill(const rba_store* st, const void* q, int32_t n_chun
   a.store_batch = d.batch;
   a.staged = p.staged ? 1 : 0;
   a.n_att_max = p.n_att_max;
+  a.od = d.head_dim;
   a.scale_log2 = scale * 1.4426950408889634f;
 
   __nv_bfloat16* SK = nullptr;
   __nv_bfloat16* SV = nullptr;
   if (p.staged) {
     SK = static_cast<__nv_bfloat16*>(workspace);
-    SV = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + p.ws_bytes / 2);
+    SV = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + p.staged_bytes / 2);
     const size_t gsmem = size_t(2 * k + 5) * sizeof(int);
     if (gsmem > 200 * 1024) return RBA_ERR_UNSUPPORTED;
     RBA_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(gather_kernel), gsmem));
@@ -786,6 +813,27 @@ rba_status rba_attend_prefill(const rba_store* st, const void* q, int32_t n_chun
   CUtensorMap mq, mpk, mpv, msk, msv, mck, mcv;
   const int64_t pool_rows = int64_t(d.batch) * d.n_kv_heads * d.capacity_tokens;
   const int64_t chunk_rows = int64_t(n_chunks) * d.n_kv_heads * chunk_len;
+  if (p.padded) {
+    char* base = static_cast<char*>(workspace) + p.staged_bytes;
+    void* qp = base;
+    void* kp = base + p.q_pad;
+    void* vp = base + p.q_pad + p.kv_pad;
+    const int64_t q_rows = int64_t(n_chunks) * d.n_q_heads * chunk_len;
+    const int words = d.head_dim / 2;
+    auto pad = [&](const void* src, void* dst, int64_t rows) {
+      int64_t grid = (rows * (kHD / 2) + 255) / 256;
+      if (grid > int64_t(num_sms()) * 16) grid = int64_t(num_sms()) * 16;
+      pad_rows_kernel<<<static_cast<int>(grid), 256, 0, stream>>>(
+          static_cast<const uint32_t*>(src), static_cast<uint32_t*>(dst), rows, words);
+    };
+    pad(q, qp, q_rows);
+    pad(chunk_k, kp, chunk_rows);
+    pad(chunk_v, vp, chunk_rows);
+    RBA_LAUNCH_CHECK();
+    q = qp;
+    chunk_k = kp;
+    chunk_v = vp;
+  }
   if (!make_map(&mq, q, int64_t(n_chunks) * d.n_q_heads * chunk_len) ||
       !make_map(&mpk, st->k, pool_rows) || !make_map(&mpv, st->v, pool_rows) ||
       !make_map(&mck, chunk_k, chunk_rows) || !make_map(&mcv, chunk_v, chunk_rows))
@@ -814,12 +862,11 @@ size_t rba_attend_prefill_workspace_size(const rba_store* st, int32_t n_chunks,
                                          int32_t chunk_len, int32_t n_sel, int32_t k, int64_t T,
                                          int32_t sink, int32_t window) {
   using namespace rba;
-  (void)chunk_len;
   (void)n_sel;
   rba::Geometry g;
   if (st == nullptr || n_chunks <= 0 || k < 0 || geometry(st, T, sink, window, &g) != RBA_OK)
     return 0;
-  return plan(st, g, n_chunks, k).ws_bytes;
+  return plan(st, g, n_chunks, chunk_len, k).ws_bytes;
 }
 
 }  // extern "C"

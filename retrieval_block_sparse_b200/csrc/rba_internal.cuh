@@ -11,6 +11,7 @@
 
 struct rba_store {
   rba_store_desc d;
+  int32_t pitch;          // elements per row of the K/V and representation pools (64 or 128)
   void* k;
   void* v;
   void* rep;
@@ -18,6 +19,7 @@ struct rba_store {
   int32_t* status;
   int64_t cap_blocks;
   int32_t score_reduce;   // rba_score_reduce: how a block's r representative keys combine
+  unsigned long long wait_ns;  // bound of the one-launch decode step's waits (ns)
 };
 
 namespace rba {
@@ -33,6 +35,7 @@ enum Where : int32_t {
   kWherePrefill = 5,
   kWhereFused = 6,
   kWhereMemory = 7,
+  kWhereStep = 8,
 };
 
 __device__ __forceinline__ void report(int32_t* status, int32_t code, int32_t where,
@@ -114,6 +117,9 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // ---------------------------------------------------------------------------
 // host side
 
+// Default bound of a device-side wait (a store's wait limit until changed).
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+
 struct Geometry {
   int64_t T;
   int32_t bs;
@@ -131,6 +137,10 @@ int num_sms();
 // Raises a kernel's dynamic shared-memory limit once per (device, kernel);
 // later calls (including inside stream capture) make no CUDA call.
 cudaError_t ensure_smem(const void* kernel, size_t bytes);
+// CTAs of `kernel` that fit on one SM with this block size and dynamic shared
+// memory (raising the kernel's limit first), cached per (device, kernel,
+// size); -1 on a CUDA error.
+int occupancy(const void* kernel, int threads, size_t smem);
 
 #define RBA_CUDA_TRY(expr)                          \
   do {                                              \
@@ -154,5 +164,11 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // or rejects the arguments.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows);
 inline size_t dtype_size(rba_dtype t) { return t == RBA_BF16 ? 2 : 4; }
+// Row pitch (elements) of the pools for a head dim: 64 up to 64, else 128;
+// -1 for head dims the library does not hold (not a multiple of 4, or > 128).
+inline int32_t pool_pitch(int32_t head_dim) {
+  if (head_dim < 4 || head_dim > 128 || head_dim % 4 != 0) return -1;
+  return head_dim <= 64 ? 64 : 128;
+}
 
 }  // namespace rba

@@ -52,6 +52,23 @@ __global__ void __launch_bounds__(kQsumThreads) qsum_kernel(const QT* __restrict
   }
 }
 
+// qsum for q rows of qd < D elements (head dims below the pools' row pitch):
+// one thread per column, rows summed in order; columns past qd are zero.
+template <typename QT>
+__global__ void qsum_rows_kernel(const QT* __restrict__ q, float* __restrict__ qsum, int Hq,
+                                 int Hkv, int n_q, int qd, int D) {
+  const int bh = blockIdx.x;
+  const int b = bh / Hkv, h = bh % Hkv, g = Hq / Hkv;
+  const int64_t rows = int64_t(g) * n_q;
+  const QT* base = q + (int64_t(b) * Hq + h * g) * n_q * qd;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    if (d < qd)
+      for (int64_t r = 0; r < rows; ++r) acc += Elem<QT>::to_f32(base[r * qd + d]);
+    qsum[int64_t(bh) * D + d] = acc;
+  }
+}
+
 __global__ void score_cos_kernel(const float* __restrict__ qe, const float* __restrict__ bank,
                                  float* __restrict__ scores, int d_ret, int first, int nc) {
   extern __shared__ float sq[];
@@ -91,6 +108,18 @@ rba_status launch_qsum(const rba_store* st, const void* q, int n_q, float* qsum,
                        cudaStream_t stream) {
   const rba_store_desc& d = st->d;
   const int BH = d.batch * d.n_kv_heads;
+  if (d.head_dim != st->pitch) {
+    if (d.dtype == RBA_BF16)
+      qsum_rows_kernel<__nv_bfloat16><<<BH, st->pitch, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(q), qsum, d.n_q_heads, d.n_kv_heads, n_q, d.head_dim,
+          st->pitch);
+    else
+      qsum_rows_kernel<float><<<BH, st->pitch, 0, stream>>>(
+          static_cast<const float*>(q), qsum, d.n_q_heads, d.n_kv_heads, n_q, d.head_dim,
+          st->pitch);
+    RBA_LAUNCH_CHECK();
+    return RBA_OK;
+  }
 #define RBA_QSUM(QT_, D_)                                                                \
   qsum_kernel<QT_, D_><<<BH, kQsumThreads, 0, stream>>>(static_cast<const QT_*>(q), qsum, \
                                                          d.n_q_heads, d.n_kv_heads, n_q)
@@ -123,6 +152,7 @@ rba_status launch_score_dot(const rba_store* st, const void* q, int n_q, const f
   a.n_q = n_q;
   a.first = g.first;
   a.nc = g.nc;
+  a.qd = d.head_dim;
   a.max_over_keys = st->score_reduce == RBA_SCORE_MAX;
   if (d.mode == RBA_REP_IDENTITY) {
     a.rep = st->k;
@@ -132,7 +162,7 @@ rba_status launch_score_dot(const rba_store* st, const void* q, int n_q, const f
     a.rep_rows = st->cap_blocks;
   }
   const bool rep_f32 = d.mode == RBA_REP_MEAN || d.dtype == RBA_F32;
-  return dispatch_score_dot(a, d.dtype == RBA_BF16, rep_f32, d.head_dim, d.n_rep, BH, stream);
+  return dispatch_score_dot(a, d.dtype == RBA_BF16, rep_f32, st->pitch, d.n_rep, BH, stream);
 }
 
 rba_status launch_score_cos(const rba_store* st, const float* qe, int n_q, const Geometry& g,

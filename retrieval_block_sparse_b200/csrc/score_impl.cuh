@@ -12,6 +12,7 @@ struct ScoreArgs {
   const float* qsum;    // [B*Hkv][D] or nullptr
   float* scores;        // [B*Hkv][nc]
   int Hq, Hkv, n_q, first, nc;
+  int qd;               // row length of q (the rep rows hold D >= qd elements, the rest zero)
   bool max_over_keys;   // block score = max over its keys (else their sum)
 };
 
@@ -60,11 +61,11 @@ __global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int can
     float acc = 0.f;
     if (a.qsum != nullptr) {
       acc = a.qsum[int64_t(bh) * D + d];
-    } else {
+    } else if (d < a.qd) {
       const QT* q = static_cast<const QT*>(a.q);
       for (int i = 0; i < g; ++i)
         for (int t = 0; t < a.n_q; ++t)
-          acc += Elem<QT>::to_f32(q[((int64_t(b) * a.Hq + h * g + i) * a.n_q + t) * D + d]);
+          acc += Elem<QT>::to_f32(q[((int64_t(b) * a.Hq + h * g + i) * a.n_q + t) * a.qd + d]);
     }
     qs[d] = acc;
   }

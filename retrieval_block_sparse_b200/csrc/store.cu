@@ -70,6 +70,32 @@ cudaError_t ensure_smem(const void* kernel, size_t bytes) {
   return e;
 }
 
+int occupancy(const void* kernel, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::unordered_map<uint64_t, int> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const uint64_t key = reinterpret_cast<uint64_t>(kernel) ^ (uint64_t(dev) << 56) ^
+                       (uint64_t(smem) << 20) ^ uint64_t(threads);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find(key);
+    if (it != done.end()) return it->second;
+  }
+  if (ensure_smem(kernel, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  done[key] = occ;
+  return occ;
+}
+
 }  // namespace rba
 
 extern "C" {
@@ -82,7 +108,7 @@ rba_status rba_store_create(const rba_store_desc* d, void* k_pool, void* v_pool,
       d->n_rep <= 0 || d->capacity_tokens <= 0 || d->n_q_heads % d->n_kv_heads != 0)
     return RBA_ERR_INVALID_ARG;
   if (d->dtype != RBA_F32 && d->dtype != RBA_BF16) return RBA_ERR_INVALID_ARG;
-  if (d->head_dim != 64 && d->head_dim != 128) return RBA_ERR_UNSUPPORTED;
+  if (rba::pool_pitch(d->head_dim) < 0) return RBA_ERR_UNSUPPORTED;
   if (k_pool == nullptr || v_pool == nullptr) return RBA_ERR_INVALID_ARG;
   if (d->capacity_tokens >= (int64_t(1) << 31)) return RBA_ERR_INVALID_ARG;
   switch (d->mode) {
@@ -111,6 +137,7 @@ rba_status rba_store_create(const rba_store_desc* d, void* k_pool, void* v_pool,
   rba_store* s = new (std::nothrow) rba_store;
   if (s == nullptr) return RBA_ERR_INVALID_ARG;
   s->d = *d;
+  s->pitch = rba::pool_pitch(d->head_dim);
   s->k = k_pool;
   s->v = v_pool;
   s->rep = rep_pool;
@@ -118,6 +145,7 @@ rba_status rba_store_create(const rba_store_desc* d, void* k_pool, void* v_pool,
   s->status = status_word;
   s->cap_blocks = d->capacity_tokens / d->block_size;
   s->score_reduce = RBA_SCORE_SUM;
+  s->wait_ns = rba::kDefaultWaitNs;
   *out = s;
   return RBA_OK;
 }
@@ -151,6 +179,8 @@ rba_status rba_store_check(const rba_store* store, cudaStream_t stream) {
   return RBA_OK;
 }
 
+int32_t rba_row_pitch(int32_t head_dim) { return rba::pool_pitch(head_dim); }
+
 const char* rba_status_string(rba_status s) {
   switch (s) {
     case RBA_OK: return "ok";
@@ -167,6 +197,12 @@ const char* rba_status_string(rba_status s) {
 int32_t rba_version(void) { return 100; }
 
 }  // extern "C"
+
+extern "C" rba_status rba_store_set_wait_limit_ns(rba_store* st, uint64_t ns) {
+  if (st == nullptr) return RBA_ERR_INVALID_ARG;
+  st->wait_ns = ns == 0 ? rba::kDefaultWaitNs : ns;
+  return RBA_OK;
+}
 
 extern "C" rba_status rba_store_set_score_reduce(rba_store* st, int32_t reduce) {
   if (st == nullptr || (reduce != RBA_SCORE_SUM && reduce != RBA_SCORE_MAX))

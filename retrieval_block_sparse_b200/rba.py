@@ -28,6 +28,7 @@ SIGNATURES = {
     "rba_store_create": (_c_i32, [_p, _p, _p, _p, _p, _p, ctypes.POINTER(_p)]),
     "rba_store_destroy": (_c_i32, [_p]),
     "rba_store_set_score_reduce": (_c_i32, [_p, _c_i32]),
+    "rba_store_set_wait_limit_ns": (_c_i32, [_p, ctypes.c_uint64]),
     "rba_candidates": (_c_i32, [_p, _c_i64, _c_i32, _c_i32, ctypes.POINTER(_c_i32),
                                 ctypes.POINTER(_c_i32)]),
     "rba_memorize": (_c_i32, [_p, _p, _p, _c_i64, _c_i32, _p, _c_i32, _c_f32, _p]),
@@ -39,6 +40,8 @@ SIGNATURES = {
     "rba_attend_workspace_size": (_c_size, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
     "rba_attend_noalloc": (_c_i32, [_p, _p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32, _p, _p,
                                     _p]),
+    "rba_attend_landmark_gated": (_c_i32, [_p, _p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32,
+                                           _p, _p, _p]),
     "rba_attend_prefill": (_c_i32, [_p, _p, _c_i32, _c_i32, _p, _c_i32, _c_i32, _c_i64, _c_i32,
                                     _c_i32, _p, _p, _c_f32, _p, _p, _p, _c_size, _p]),
     "rba_attend_prefill_workspace_size": (_c_size, [_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i64,
@@ -50,6 +53,11 @@ SIGNATURES = {
     "rba_decode_step_launches": (_c_i32, [_p, _c_i32, _c_i64, _c_i32, _c_i32]),
     "rba_stream_step": (_c_i32, [_p, _p, _p, _p, _c_i64, _c_i32, _c_i32, _c_i32, _c_f32, _p,
                                  _c_i32, _p, _p, _p, ctypes.POINTER(_c_i32), _p, _c_size, _p]),
+    "rba_group_means": (_c_i32, [_p, _c_i64, _c_i32, _c_i32, _p, _p]),
+    "rba_approx_select": (_c_i32, [_p, _p, _c_i64, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _p,
+                                   _p, _p, _p, _p, _c_size, _p]),
+    "rba_approx_select_workspace_size": (_c_size, [_p, _c_i64, _c_i32, _c_i32, _c_i32, _c_i32,
+                                                   _c_i32]),
     "rba_memory_rule": (_c_i32, [_c_i64, ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i64),
                                  ctypes.POINTER(_c_i64)]),
     "rba_memory_units": (_c_i32, [_p]),
@@ -59,6 +67,7 @@ SIGNATURES = {
     "rba_decode_step_host": (_c_i32, [_p, _p, _p, _c_i32, _c_i64, _c_i32, _c_i32, _c_f32, _p, _p,
                                       _p, _p, _p, _p, _p, _c_size, _p]),
     "rba_store_check": (_c_i32, [_p, _p]),
+    "rba_row_pitch": (_c_i32, [_c_i32]),
     "rba_status_string": (ctypes.c_char_p, [_c_i32]),
     "rba_version": (_c_i32, []),
 }
@@ -126,10 +135,12 @@ class _Desc(ctypes.Structure):
 class Store:
     """A block store: caller-owned device pools described to the library.
 
-    Pools (allocated here with torch, owned by this object):
-      k, v     [B][Hkv][capacity][D]         store dtype
-      rep      mean: fp32 [B][Hkv][cap_blocks][1][D]; topr_attn / external:
-               dtype [B][Hkv][cap_blocks][r][D]; embed_cosine: fp32
+    Pools (allocated here with torch, owned by this object), rows of P =
+    rba_row_pitch(D) elements (P = D for D = 64 or 128; else the first D are
+    the row and the rest stay zero -- write rows through `kv_rows`):
+      k, v     [B][Hkv][capacity][P]         store dtype
+      rep      mean: fp32 [B][Hkv][cap_blocks][1][P]; topr_attn / external:
+               dtype [B][Hkv][cap_blocks][r][P]; embed_cosine: fp32
                [B][cap_blocks][d_ret]; identity: none
       rep_pos  int32 [B][Hkv][cap_blocks][r] (topr_attn)
       status   int32[4] device status word
@@ -144,17 +155,22 @@ class Store:
         self.B, self.Hq, self.Hkv, self.D = batch, n_q_heads, n_kv_heads, head_dim
         self.bs, self.r, self.d_ret, self.cap = block_size, n_rep, d_ret, capacity_tokens
         self.cap_blocks = capacity_tokens // block_size
+        # pool rows hold `pitch` elements: the head dim, then zero padding
+        self.pitch = lib().rba_row_pitch(head_dim)
+        if self.pitch < 0:
+            raise RbaError(ERR_UNSUPPORTED, f"head_dim {head_dim}")
+        P = self.pitch
         td = _tdtype(self.dtype)
         dev = torch.device(device)
-        self.k = torch.zeros((batch, n_kv_heads, capacity_tokens, head_dim), dtype=td, device=dev)
+        self.k = torch.zeros((batch, n_kv_heads, capacity_tokens, P), dtype=td, device=dev)
         self.v = torch.zeros_like(self.k)
         self.rep = None
         self.rep_pos = None
         if mode == "mean":
-            self.rep = torch.zeros((batch, n_kv_heads, self.cap_blocks, 1, head_dim),
+            self.rep = torch.zeros((batch, n_kv_heads, self.cap_blocks, 1, P),
                                    dtype=torch.float32, device=dev)
         elif mode in ("topr_attn", "external"):
-            self.rep = torch.zeros((batch, n_kv_heads, self.cap_blocks, n_rep, head_dim), dtype=td,
+            self.rep = torch.zeros((batch, n_kv_heads, self.cap_blocks, n_rep, P), dtype=td,
                                    device=dev)
             if mode == "topr_attn":
                 self.rep_pos = torch.full((batch, n_kv_heads, self.cap_blocks, n_rep), -1,
@@ -176,6 +192,11 @@ class Store:
                    "rba_store_set_score_reduce")
         self.score_reduce = score_reduce
 
+    def set_wait_limit_ns(self, ns):
+        """Bound of the one-launch decode step's device waits (0: the default 2 s)."""
+        _check(lib().rba_store_set_wait_limit_ns(self.handle, int(ns)),
+               "rba_store_set_wait_limit_ns")
+
     def __del__(self):
         h = getattr(self, "handle", None)
         if h is not None and _LIB is not None:
@@ -185,6 +206,10 @@ class Store:
     @property
     def tdtype(self):
         return _tdtype(self.dtype)
+
+    def kv_rows(self, t):
+        """The first D elements of every row of a pool tensor (a view to write into)."""
+        return t[..., :self.D]
 
     # -- geometry ------------------------------------------------------------
     def candidates(self, T, sink, window):
@@ -244,6 +269,21 @@ class Store:
                                 _stream()), "rba_attend")
         return out, lse
 
+    def attend_gated(self, q, idx, T, sink, window, *, scale=None, out=None, lse=None):
+        """Landmark-gated attention (landmark stores): each retrieved block enters
+        the softmax once, with its landmark's logit (see rba.h)."""
+        k = idx.shape[-1] if idx is not None else 0
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.D)
+        if out is None:
+            out = torch.empty((self.B, self.Hq, self.D), dtype=torch.float32, device=q.device)
+        if lse is None:
+            lse = torch.empty((self.B, self.Hq), dtype=torch.float32, device=q.device)
+        _check(lib().rba_attend_landmark_gated(self.handle, _ptr(q), _ptr(idx), k, T, sink,
+                                               window, scale, _ptr(out), _ptr(lse), _stream()),
+               "rba_attend_landmark_gated")
+        return out, lse
+
     def prefill_workspace(self, n_chunks, chunk_len, n_sel, k, T, sink, window):
         n = lib().rba_attend_prefill_workspace_size(self.handle, n_chunks, chunk_len, n_sel, k, T,
                                                     sink, window)
@@ -273,9 +313,10 @@ class Store:
         return torch.zeros(max(n, 16), dtype=torch.uint8, device=self.k.device)
 
     def decode_plan(self, k, T, sink, window):
-        """2: score -> top-k -> whole-block tensor-core attention kernel, overlapped
-        (programmatic dependent launches); 1: the same with the CUDA-core attention
-        kernel; 0: score -> top-k -> split-K in stream order; <0: see rba.h."""
+        """3: the whole step in one cooperative launch; 2: score -> top-k ->
+        whole-block tensor-core attention kernel, overlapped (programmatic
+        dependent launches); 1: the same with the CUDA-core attention kernel;
+        0: score -> top-k -> split-K in stream order; <0: see rba.h."""
         return lib().rba_decode_step_plan(self.handle, k, T, sink, window)
 
     def decode_launches(self, k, T, sink, window):
@@ -325,6 +366,42 @@ class Store:
         kk = used.value
         sel = idx.reshape(-1)[: self.B * self.Hkv * kk].reshape(self.B, self.Hkv, kk)
         return sel, out, lse
+
+    # -- two-stage approximate token retrieval (block size 1) ---------------------
+    def group_means(self, group, *, first_group=0, n_groups=None, out=None):
+        """Mean key of every group of `group` consecutive tokens (fp32 index
+        [B][Hkv][capacity // group][P]); groups [first_group, first_group + n_groups)."""
+        cap_groups = self.cap // group
+        if n_groups is None:
+            n_groups = cap_groups - first_group
+        if out is None:
+            out = torch.zeros((self.B, self.Hkv, cap_groups, self.pitch), dtype=torch.float32,
+                              device=self.k.device)
+        _check(lib().rba_group_means(self.handle, first_group, n_groups, group, _ptr(out),
+                                     _stream()), "rba_group_means")
+        return out
+
+    def approx_select(self, q, T, sink, window, group, groups_kept, k, means, *, idx=None,
+                      groups_out=None, scanned=None, workspace=None):
+        """Two-stage selection of k tokens per (batch, kv head).  Returns
+        (idx [B][Hkv][k], kept groups [B][Hkv][groups_kept], keys read [B][Hkv])."""
+        dev = q.device
+        if idx is None:
+            idx = torch.empty((self.B, self.Hkv, k), dtype=torch.int32, device=dev)
+        if groups_out is None:
+            groups_out = torch.empty((self.B, self.Hkv, groups_kept), dtype=torch.int32,
+                                     device=dev)
+        if scanned is None:
+            scanned = torch.empty((self.B, self.Hkv), dtype=torch.int32, device=dev)
+        if workspace is None:
+            n = lib().rba_approx_select_workspace_size(self.handle, T, sink, window, group,
+                                                       groups_kept, k)
+            workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+        _check(lib().rba_approx_select(self.handle, _ptr(q), T, sink, window, group,
+                                       groups_kept, k, _ptr(means), _ptr(idx), _ptr(groups_out),
+                                       _ptr(scanned), _ptr(workspace), workspace.numel(),
+                                       _stream()), "rba_approx_select")
+        return idx, groups_out, scanned
 
     # -- dynamic memory update ---------------------------------------------------
     def memory_units(self):

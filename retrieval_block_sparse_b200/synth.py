@@ -232,12 +232,15 @@ def decode_inputs(w: DecodeWorkload) -> dict:
     elif w.recipe == "drift":
         from scipy.signal import lfilter
         rho = 0.97
-        for b in range(B):
-            for h in range(Hkv):
-                z = K[b, h]
-                zi = (rho * z[0])[None, :]
-                K[b, h, 1:] = lfilter([math.sqrt(1.0 - rho * rho)], [1.0, -rho], z[1:], axis=0,
-                                      zi=zi)[0]
+
+        def drift(bh):
+            # one (batch, kv head) slice at a time; slices are independent, so
+            # the threads change no value
+            z = K[bh // Hkv, bh % Hkv]
+            zi = (rho * z[0])[None, :]
+            z[1:] = lfilter([math.sqrt(1.0 - rho * rho)], [1.0, -rho], z[1:], axis=0, zi=zi)[0]
+        with ThreadPoolExecutor(max(1, min(B * Hkv, os.cpu_count() or 1))) as ex:
+            list(ex.map(drift, range(B * Hkv)))
         q = _normal(s, "q", (B, Hq, D), mean=0.5, std=1.5)
     elif w.recipe == "planted":
         u = _unit_rows(_normal(s, "u", (Hkv, D)).astype(np.float64)).astype(np.float32)

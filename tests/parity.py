@@ -43,8 +43,8 @@ def make_decode_store(rba, w, x):
     st = rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                    head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
                    dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep)
-    st.k.copy_(dev(x["K"], w.dtype))
-    st.v.copy_(dev(x["V"], w.dtype))
+    st.kv_rows(st.k).copy_(dev(x["K"], w.dtype))  # (pool rows may be padded past D)
+    st.kv_rows(st.v).copy_(dev(x["V"], w.dtype))
     aux = None
     if w.rep_mode == "topr_attn":
         aux = dev(x["probe"], w.dtype)

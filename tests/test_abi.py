@@ -67,7 +67,12 @@ def test_store_create_validates(L):
     s, h = _create(L)
     assert s == 0 and h.value
     L.rba_store_destroy(h)
-    assert _create(L, head_dim=96)[0] == 2          # unsupported head dim
+    assert _create(L, head_dim=130)[0] == 2         # head dim above the 128-element row
+    assert _create(L, head_dim=98)[0] == 2          # not a multiple of 4
+    for hd, pitch in ((64, 64), (128, 128), (100, 128), (96, 128), (48, 64)):
+        s, h = _create(L, head_dim=hd)               # held in rows of the pitch
+        assert s == 0 and L.rba_row_pitch(hd) == pitch, hd
+        L.rba_store_destroy(h)
     assert _create(L, n_q_heads=3)[0] == 1          # Hq not a multiple of Hkv
     assert _create(L, mode=4)[0] == 1               # identity needs block size 1
     assert _create(L, mode=4, block_size=1)[0] == 0

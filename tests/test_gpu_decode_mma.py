@@ -54,7 +54,8 @@ def _prepared(name):
 def test_attend_on_oracle_selection(rba, name):
     w, x, ref = _prepared(name)
     st = make_decode_store(rba, w, x)
-    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 2  # the whole-block kernel
+    # rba_attend runs the whole-block kernel (the decode step may run in one launch)
+    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) in (2, 3)
     idx = torch.from_numpy(ref["idx"].astype(np.int32)).cuda()
     out, lse = st.attend(dev(x["q"], w.dtype), idx, w.context, w.sink, w.window)
     st.check()
