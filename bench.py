@@ -580,11 +580,13 @@ def _time_graph(g, stream, seconds, min_iters=5):
     return e0.elapsed_time(e1) / n, n
 
 
-def measure_decode_config(name, dev, seconds, pk, score_reduce="sum", workload=None):
+def measure_decode_config(name, dev, seconds, pk, score_reduce="sum", workload=None,
+                          one_launch=False):
     """Decode-step throughput of one decode config (graph-replayed steps; L2
     defeated by rotating store replicas, or by an L2-sized write between
     steps whose own time is subtracted when replicas would not fit).
-    score_reduce="max": the max-over-representative-keys score variant."""
+    score_reduce="max": the max-over-representative-keys score variant;
+    one_launch: the step as one cooperative launch where eligible."""
     import torch
     import retrieval_block_sparse_b200 as rba
     from retrieval_block_sparse_b200 import synth
@@ -592,10 +594,13 @@ def measure_decode_config(name, dev, seconds, pk, score_reduce="sum", workload=N
     x = synth.decode_inputs(w)
 
     def new_store():
-        return rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
-                         head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
-                         dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep, device=dev,
-                         score_reduce=score_reduce)
+        s = rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                      head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
+                      dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep, device=dev,
+                      score_reduce=score_reduce)
+        if one_launch:
+            s.set_decode_step_one_launch(True)
+        return s
     st = new_store()
     st.kv_rows(st.k).copy_(_to_dev(x["K"], w.dtype, dev))
     st.kv_rows(st.v).copy_(_to_dev(x["V"], w.dtype, dev))
@@ -937,6 +942,8 @@ def measure_configs(dev, seconds):
         out[name] = measure_decode_config(name, dev, seconds, pk)
     out["infllm-decode-128k:max-over-rep-keys"] = measure_decode_config(
         "infllm-decode-128k", dev, seconds, pk, score_reduce="max")
+    out["infllm-decode-128k:one-launch"] = measure_decode_config(
+        "infllm-decode-128k", dev, seconds, pk, one_launch=True)
     for name in ("memlong-cosine-prefill", "token-retrieval-prefill-1m"):
         out[name] = measure_prefill_config(name, dev, seconds, pk)
     # head dim 100 (MemLong's OpenLLaMA-3B: 32 heads of 100), pool rows padded to 128

@@ -138,6 +138,15 @@ rba_status rba_store_set_score_reduce(rba_store* store, int32_t reduce);
  * Errors: INVALID_ARG (NULL store). */
 rba_status rba_store_set_wait_limit_ns(rba_store* store, uint64_t ns);
 
+/* Whether rba_decode_step may run the whole step as one cooperative launch on this
+ * store (host only; on = 1), where rba_decode_step_plan() then reports 3; 0 (the
+ * default) keeps the three-kernel step.  On B200 the three-kernel step is the faster
+ * of the two at the 128K-token InfLLM decode shape; the one-launch step is kept for
+ * shapes and callers that prefer a single launch.  Results are the same either way
+ * (same definitions; floating-point sums may differ in rounding order).
+ * Errors: INVALID_ARG (NULL store, on not 0 or 1). */
+rba_status rba_store_set_decode_step_one_launch(rba_store* store, int32_t on);
+
 /* Candidate range for a store holding T tokens with the given sink/window
  * (host only; see the vocabulary above).  Errors: INVALID_ARG (tail block
  * outside the window, negative sizes, T > capacity). */
@@ -305,7 +314,8 @@ size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t
                                       int32_t sink, int32_t window);
 
 /* How rba_decode_step runs this problem (host only; queries the device, launches nothing):
- *   3   the whole step in one cooperative launch: bf16 store, block size a multiple of 64,
+ *   3   the whole step in one cooperative launch (only after
+ *       rba_store_set_decode_step_one_launch(store, 1)): bf16 store, block size a multiple of 64,
  *       head dim 64 or 128, GQA group of 1, 2 or 4, dot-mode representations (mean, top-r,
  *       landmark) with at most 8 keys per block, 1 <= k <= 256, at most 4096 candidates
  *       per (batch, kv head), at most half as many (batch, kv head) units as SMs, and a

@@ -53,6 +53,8 @@ struct Groups {
   static_assert(G % NGRP == 0 && kCW % NGRP == 0, "even split");
 };
 constexpr int kMaxK = 2048;                   // selected blocks per (b, kv head)
+// shared-memory table: prefix [kMaxK + 1], starts [kMaxK], sink/window [5]
+static_assert((kMaxK + 1) + kMaxK + 5 <= 2 * (kMaxK + 4), "selection table room");
 constexpr int kMinRowsPerCta = 128;           // grid shrinks for small problems
 constexpr int kMaxGrid = 256;                 // CTAs (one per SM)
 
@@ -169,7 +171,7 @@ struct FusedSmem {
   static constexpr int up16(int x) { return (x + 15) & ~15; }
   // regions after the stage ring (NS * STAGE, chosen at launch)
   static constexpr int RED = up16(kCW * G * (D + 2) * 4);       // warp states
-  static constexpr int SEL = (kMaxK + 4) * 4 * 2;               // selected prefix + starts
+  static constexpr int SEL = (kMaxK + 4) * 4 * 2;  // selected prefix + starts, sink/window table
   static constexpr int MISC = kMiscBytes;
   static size_t bytes(int NS) { return size_t(NS) * STAGE + RED + SEL + MISC; }
 };
@@ -371,15 +373,9 @@ __device__ void issue_item(const FusedArgs& a, const Item& item, char* stg, uint
   const int* pref;
   const int* phys;
   int nseg;
-  int st_pref[3], st_phys[2];
   if (item.kind == 1) {
-    st_pref[0] = 0;
-    st_pref[1] = a.at.sink_end;
-    st_pref[2] = a.L_st;
-    st_phys[0] = 0;
-    st_phys[1] = static_cast<int>(a.at.w0);
-    pref = st_pref;
-    phys = st_phys;
+    pref = sel_phys + kMaxK;  // the sink/window table (written by produce)
+    phys = pref + 3;
     nseg = 2;
   } else {
     if (item.bh != *sel_bh) {
@@ -471,6 +467,19 @@ template <class Geo>
 __device__ __forceinline__ void produce(const FusedArgs& a, char* stages, uint64_t* full,
                                         uint64_t* empty, Meta* meta, int* sel_pref,
                                         int* sel_phys, volatile int* abort_flag) {
+  // the sink/window segments (prefix 0, sink_end, L_st; first rows 0, w0),
+  // in shared memory after the selection's table: a small array indexed at
+  // run time would live in local memory, and every access would wait on an
+  // L2 kept busy by the copies
+  if ((threadIdx.x & 31) == 0) {
+    int* st_tab = sel_phys + kMaxK;
+    st_tab[0] = 0;
+    st_tab[1] = a.at.sink_end;
+    st_tab[2] = a.L_st;
+    st_tab[3] = 0;
+    st_tab[4] = static_cast<int>(a.at.w0);
+  }
+  __syncwarp();
   const int NS = a.NS;
   Iter it;
   iter_begin(a, it);
@@ -662,7 +671,7 @@ struct MmaSmem {
   static constexpr int up16(int x) { return (x + 15) & ~15; }
   static constexpr int RED = up16(kMW * G * (D + 2) * 4);       // warp states
   static constexpr int QF = kMW * (D / 16) * 32 * 8;            // per-warp Q fragments
-  static constexpr int SEL = (kMaxK + 4) * 4 * 2;               // selected prefix + starts
+  static constexpr int SEL = (kMaxK + 4) * 4 * 2;  // selected prefix + starts, sink/window table
   static constexpr int MISC = kMiscBytes;
   static constexpr int ALIGN = 1024;                            // ring base alignment slack
   static size_t bytes(int NS) {
@@ -681,6 +690,19 @@ __device__ __forceinline__ void produce_pieces(const FusedArgs& a, const CUtenso
                                                int* sel_phys) {
   using Geo = MmaGeo<D>;
   const int lane = threadIdx.x & 31;
+  // the sink/window segments (prefix 0, sink_end, L_st; first rows 0, w0),
+  // in shared memory after the selection's table: a small array indexed at
+  // run time would live in local memory, and every access would wait on an
+  // L2 kept busy by the copies
+  if ((threadIdx.x & 31) == 0) {
+    int* st_tab = sel_phys + kMaxK;
+    st_tab[0] = 0;
+    st_tab[1] = a.at.sink_end;
+    st_tab[2] = a.L_st;
+    st_tab[3] = 0;
+    st_tab[4] = static_cast<int>(a.at.w0);
+  }
+  __syncwarp();
   const int NS = a.NS;
   int j = 0, s = 0, sel_bh = -1;
   uint32_t ph = 0;
@@ -727,18 +749,12 @@ __device__ __forceinline__ void produce_pieces(const FusedArgs& a, const CUtenso
       int v = kind == 1 ? s0 : sel0;
       const int vend = kind == 1 ? s1 : sel1;
       if (v >= vend) continue;
-      int st_pref[3], st_phys[2];
       const int* pref;
       const int* phys;
       int nseg;
       if (kind == 1) {
-        st_pref[0] = 0;
-        st_pref[1] = a.at.sink_end;
-        st_pref[2] = a.L_st;
-        st_phys[0] = 0;
-        st_phys[1] = static_cast<int>(a.at.w0);
-        pref = st_pref;
-        phys = st_phys;
+        pref = sel_phys + kMaxK;  // the sink/window table
+        phys = pref + 3;
         nseg = 2;
       } else {
         if (!selection_visible) {
@@ -820,8 +836,10 @@ __global__ void __launch_bounds__(kMFT, 1)
   using Geo = MmaGeo<D>;
   using S = MmaSmem<D, G>;
   extern __shared__ char smem_raw[];
-  char* stages = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                         ~uintptr_t(1023));
+  // 1024-byte aligned base, offset from the shared array itself (an integer
+  // round trip would hide from the compiler that the pointers address shared
+  // memory and turn every access into a generic one)
+  char* stages = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int NS = a.NS;
   float* red = reinterpret_cast<float*>(stages + size_t(NS) * Geo::STAGE);
   uint2* qfrag = reinterpret_cast<uint2*>(reinterpret_cast<char*>(red) + S::RED);

@@ -21,7 +21,7 @@
 //     (mma.sync, as the whole-block attention kernel);
 //   * selector warp: waits until every part of the head has published its
 //     scores, reads the head's scores and selects the top k with one warp
-//     (value-binned histogram, exact radix select where that does not apply);
+//     (bitwise radix select on keys held in registers);
 //     every part of the head selects the same set, so no second exchange is
 //     needed.  Part 0 writes the selection out.
 // Each part's softmax state goes to a slot; the last part of the head to
@@ -103,11 +103,6 @@ __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
 // (a plain intrinsic: the compiler may issue many of these before their uses;
 // the acquire that orders them is a volatile asm with a memory clobber)
 __device__ __forceinline__ float ld_cg_f32(const float* p) { return __ldcg(p); }
-__device__ __forceinline__ unsigned lanemask_lt() {
-  unsigned m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
 
 // ---------------------------------------------------------------------------
 // scoring of one part's candidate slice (compute warps)
@@ -161,237 +156,250 @@ __device__ __forceinline__ void score_slice(const char* rep, int ns, int R, bool
 // ---------------------------------------------------------------------------
 // one-warp top-k (selector)
 //
-// The k best positions of s[0, n) under (larger score first, equal scores ->
-// lower position first), written ascending to pos[0, k).  Value binning,
-// refined: a pass histograms the current members over 256 bins linear in
-// their value range; members of the bins above the one holding the kk-th
-// largest are selected, the members of that bin stay members (compacted in
-// position order) and the rest are dropped.  A pass shrinks the range 256-fold,
-// so a few passes leave at most 32 members (ranked exactly) or members of one
-// value (the lowest positions taken).  Non-finite scores take an exact radix
-// select on the order-preserving bits instead.
-// Scratch: hist[256], cand[n] (member positions), words[(n + 31) / 32] (a bit
-// per selected position).
+// The k best positions of a head's n scores under (larger score first, equal
+// scores -> lower position first), written ascending to pos[0, k).  Scores
+// become order-preserving 32-bit keys (-0 == +0; infinities and NaNs keep the
+// order of their bits).  The scores are copied to shared memory (coalesced,
+// 32 loads in flight per lane); per chunk of 1024 positions lane l holds the
+// keys of positions [1024 c + 32 l, +32) in registers (read rotated, so the
+// 32 lanes hit 32 banks), and its selection bits of those positions form one
+// word, so the ascending positions come from one scan over the lanes.
+// A radix select finds the threshold tau two bits at a time, starting below
+// the bits that the smallest and largest keys share: the three trial values
+// of the next two bits are counted with independent compares and three warp
+// reductions, and the largest one that at least k keys reach is kept.  Once
+// at most 256 keys reach tau, they alone can reach a later trial value: they
+// are compacted to 8 registers per lane.  The search stops as soon as exactly
+// k keys reach tau; otherwise tau ends as the k-th largest key and its lowest
+// positions fill the set.
 
-struct WarpTopkSmem {
-  uint32_t* hist;
-  int* cand;
-  uint32_t* words;
-};
+constexpr int kSelRegs = 32;   // keys per lane of one 1024-position chunk
+constexpr int kSelLive = 8;    // keys per lane once at most 256 reach tau
+// (the live keys and the spare words use the positions and prefix scratch)
+static_assert(kSelLive * 32 + 32 <= 2 * kStepMaxK + 2, "live key scratch");
 
-// positions of the set bits of words[0, nw), ascending
-__device__ __forceinline__ void write_positions(const uint32_t* words, int nw, int* pos) {
+template <int N>
+__device__ __forceinline__ void count3(const uint32_t (&key)[N], uint32_t t1, uint32_t t2,
+                                       uint32_t t3, int& c1, int& c2, int& c3) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    c1 += key[i] >= t1;
+    c2 += key[i] >= t2;
+    c3 += key[i] >= t3;
+  }
+}
+
+// keys of lane l in chunk c: register i holds position 1024 c + 32 l +
+// ((i + l) & 31); positions past n read as 0 (every trial value is >= 1)
+__device__ __forceinline__ void chunk_keys(const float* sm, int n, int c, uint32_t (&key)[kSelRegs]) {
   const int lane = threadIdx.x & 31;
-  int written = 0;
-  for (int w0 = 0; w0 < nw; w0 += 32) {
-    const int w = w0 + lane;
-    uint32_t word = w < nw ? words[w] : 0u;
-    const int cnt = __popc(word);
-    int incl = cnt;
+  const int base = c * (kSelRegs * 32) + lane * 32;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    int p = written + incl - cnt;
-    while (word) {
-      const int b = __ffs(word) - 1;
-      pos[p++] = w * 32 + b;
-      word &= word - 1;
-    }
-    written += __shfl_sync(0xffffffffu, incl, 31);
+  for (int i = 0; i < kSelRegs; ++i) {
+    const int p = base + ((i + lane) & 31);
+    key[i] = ordered_f32(sm[min(p, n - 1)]) & (0u - uint32_t(p < n));
   }
-  __syncwarp();
 }
 
-// hist[bin] += 1 for every lane with `in`; lanes with the same bin add once
-__device__ __forceinline__ void hist_add(uint32_t* hist, int bin, bool in) {
-  const unsigned act = __ballot_sync(0xffffffffu, in);
-  const unsigned same = __match_any_sync(0xffffffffu, in ? bin : -1) & act;
-  if (in && int(threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], uint32_t(__popc(same)));
-}
-
-// the bin (of 256 counters, lane l holding [8 l, 8 l + 8)) that holds the
-// kk-th largest counted element; counts above it in *above, its count in *cnt
-__device__ __forceinline__ int boundary_bin(const uint32_t* hist, int kk, int* above_out,
-                                            int* cnt_out) {
-  const int lane = threadIdx.x & 31;
-  uint32_t c[8], tot = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    c[i] = hist[lane * 8 + i];
-    tot += c[i];
-  }
-  uint32_t incl = tot;  // sum over lanes >= this one
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_down_sync(0xffffffffu, incl, o);
-    if (lane + o < 32) incl += t;
-  }
-  uint32_t above = incl - tot;
-  int bin = -1, ab = 0, cn = 0;
-#pragma unroll
-  for (int i = 7; i >= 0; --i) {
-    if (above < uint32_t(kk) && uint32_t(kk) <= above + c[i]) {
-      bin = lane * 8 + i;
-      ab = static_cast<int>(above);
-      cn = static_cast<int>(c[i]);
-    }
-    above += c[i];
-  }
-  const unsigned who = __ballot_sync(0xffffffffu, bin >= 0);
-  const int src = who ? __ffs(who) - 1 : 0;
-  *above_out = __shfl_sync(0xffffffffu, ab, src);
-  *cnt_out = __shfl_sync(0xffffffffu, cn, src);
-  return __shfl_sync(0xffffffffu, bin, src);
-}
-
-__device__ __forceinline__ int value_bin256(float x, float lo, float scale) {
-  const float t = __fmul_rn(__fsub_rn(x, lo), scale);
-  return min(255, static_cast<int>(t));
-}
-
-// Exact radix select on the order-preserving score bits (4 passes of 8 bits),
-// then every larger key and the lowest-positioned equal ones.
-__device__ void warp_topk_radix(const float* s, int n, int k, int* pos, const WarpTopkSmem& w) {
-  const int lane = threadIdx.x & 31;
-  uint32_t prefix = 0, mask = 0;
-  int kk = k;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) w.hist[b] = 0u;
-    __syncwarp();
-    for (int base = 0; base < n; base += 32) {
-      const int j = base + lane;
-      const uint32_t u = j < n ? ordered_f32(s[j]) : 0u;
-      hist_add(w.hist, int((u >> shift) & 255u), j < n && (u & mask) == prefix);
-    }
-    __syncwarp();
-    int above, cnt;
-    const int d = boundary_bin(w.hist, kk, &above, &cnt);
-    __syncwarp();
-    prefix |= uint32_t(d) << shift;
-    mask |= 255u << shift;
-    kk -= above;
-  }
-  // kk of the keys equal to `prefix` are taken, lowest positions first
-  for (int base = 0; base < n; base += 32) {
-    const int j = base + lane;
-    const uint32_t u = j < n ? ordered_f32(s[j]) : 0u;
-    const unsigned gt = __ballot_sync(0xffffffffu, j < n && u > prefix);
-    const unsigned eq = __ballot_sync(0xffffffffu, j < n && u == prefix);
-    const bool mine = j < n && u == prefix && __popc(eq & lanemask_lt()) < kk;
-    const unsigned taken = __ballot_sync(0xffffffffu, mine);
-    kk -= __popc(taken);
-    if (lane == 0) w.words[base >> 5] = gt | taken;
-  }
-  __syncwarp();
-  write_positions(w.words, (n + 31) >> 5, pos);
-}
-
-__device__ void warp_topk(const float* s, int n, int k, int* pos, const WarpTopkSmem& w) {
+// g: the head's n scores in global memory; sm: shared scratch of n floats;
+// live_sm: shared scratch of 256 + 32 words
+__device__ __forceinline__ void warp_topk(const float* g, float* sm, uint32_t* live_sm, int n,
+                                          int k, int* pos) {
   const int lane = threadIdx.x & 31;
   if (k >= n) {
     for (int j = lane; j < n; j += 32) pos[j] = j;
     __syncwarp();
     return;
   }
-  const int nw = (n + 31) >> 5;
-  float lo = INFINITY, hi = -INFINITY;
-  bool bad = false;
-  for (int j = lane; j < n; j += 32) {
-    const float v = s[j];
-    bad |= !isfinite(v);
-    lo = fminf(lo, v);
-    hi = fmaxf(hi, v);
-  }
-  if (__any_sync(0xffffffffu, bad)) {
-    warp_topk_radix(s, n, k, pos, w);
-    return;
-  }
+  for (int base = 0; base < n; base += kSelRegs * 32) {
+    float v[kSelRegs];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    for (int u = 0; u < kSelRegs; ++u) v[u] = ld_cg_f32(g + min(base + u * 32 + lane, n - 1));
+#pragma unroll
+    for (int u = 0; u < kSelRegs; ++u)
+      if (base + u * 32 + lane < n) sm[base + u * 32 + lane] = v[u];
   }
-  for (int x = lane; x < nw; x += 32) w.words[x] = 0u;
   __syncwarp();
-  // members: positions [0, n) in the first pass, cand[0, nm) after it
-  int nm = n, kk = k;
-  bool first = true;
-  for (int pass = 0;; ++pass) {
-    const float scale = 256.f / (hi - lo);
-    if (!(hi > lo) || nm <= 32 || pass >= 6 || !isfinite(scale)) {
-      if (!(hi > lo)) {
-        // members of one value: the kk lowest positions
-        for (int i = lane; i < kk; i += 32) {
-          const int j = first ? i : w.cand[i];
-          atomicOr(&w.words[j >> 5], 1u << (j & 31));
-        }
-      } else {
-        // exact ranks among the members
-        for (int i = lane; i < nm; i += 32) {
-          const int j = first ? i : w.cand[i];
-          const float x = s[j];
-          int rank = 0;
-          for (int t = 0; t < nm; ++t) {
-            const int jt = first ? t : w.cand[t];
-            const float y = s[jt];
-            rank += (y > x) || (y == x && jt < j);
+  const int nch = (n + kSelRegs * 32 - 1) / (kSelRegs * 32);
+  uint32_t key0[kSelRegs];
+  chunk_keys(sm, n, 0, key0);
+  // smallest and largest key (padding keys: 0, raised for the minimum)
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int c = 0; c < nch; ++c) {
+    uint32_t key[kSelRegs];
+    if (c == 0) {
+#pragma unroll
+      for (int i = 0; i < kSelRegs; ++i) key[i] = key0[i];
+    } else {
+      chunk_keys(sm, n, c, key);
+    }
+    const int cb = c * (kSelRegs * 32) + lane * 32;
+#pragma unroll
+    for (int i = 0; i < kSelRegs; ++i) {
+      kmin = min(kmin, key[i] | (0u - uint32_t(cb + ((i + lane) & 31) >= n)));
+      kmax = max(kmax, key[i]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  // every key lies in [kmin, kmax]: the bits above their highest differing
+  // bit are common, and all n keys reach that prefix
+  uint32_t tau = kmin;
+  int cnt = n;
+  bool compact = false;
+  uint32_t live[kSelLive];
+#pragma unroll
+  for (int j = 0; j < kSelLive; ++j) live[j] = 0u;
+  const uint32_t diff = kmin ^ kmax;
+  if (diff != 0u) {
+    const int top = 31 - __clz(diff);
+    tau = top == 31 ? 0u : (kmax & ~((2u << top) - 1u));
+    for (int b = top; b >= 0 && cnt != k; b -= 2) {
+      if (!compact && cnt <= kSelLive * 32) {
+        // the keys >= tau, in any order, to live[] (cnt of them)
+        int off = 0;
+        for (int c = 0; c < nch; ++c) {
+          uint32_t key[kSelRegs];
+          if (c == 0) {
+#pragma unroll
+            for (int i = 0; i < kSelRegs; ++i) key[i] = key0[i];
+          } else {
+            chunk_keys(sm, n, c, key);
           }
-          if (rank < kk) atomicOr(&w.words[j >> 5], 1u << (j & 31));
+          const int cb = c * (kSelRegs * 32) + lane * 32;
+          uint32_t in = 0u;  // bit i: register i holds a key >= tau
+#pragma unroll
+          for (int i = 0; i < kSelRegs; ++i)
+            in |= (uint32_t(key[i] >= tau) & uint32_t(cb + ((i + lane) & 31) < n)) << i;
+          const int sc = __popc(in);
+          int incl = sc;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+          }
+          int o2 = off + incl - sc;
+          // every register is stored: a key that is out goes to this lane's
+          // spare word past the 256
+#pragma unroll
+          for (int i = 0; i < kSelRegs; ++i) {
+            const uint32_t b = (in >> i) & 1u;
+            live_sm[b ? o2 : kSelLive * 32 + lane] = key[i];
+            o2 += int(b);
+          }
+          off += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < kSelLive; ++j)
+          live[j] = live_sm[j * 32 + lane] & (0u - uint32_t(j * 32 + lane < off));
+        __syncwarp();
+        compact = true;
+      }
+      // the next two bits (b, b - 1), or bit 0 alone
+      const int sh = b >= 1 ? b - 1 : 0;
+      const uint32_t t1 = tau | (1u << sh);
+      const uint32_t t2 = b >= 1 ? tau | (2u << sh) : t1;
+      const uint32_t t3 = b >= 1 ? tau | (3u << sh) : t1;
+      int c1 = 0, c2 = 0, c3 = 0;
+      if (compact) {
+        count3(live, t1, t2, t3, c1, c2, c3);
+      } else {
+        count3(key0, t1, t2, t3, c1, c2, c3);
+        for (int c = 1; c < nch; ++c) {
+          uint32_t key[kSelRegs];
+          chunk_keys(sm, n, c, key);
+          count3(key, t1, t2, t3, c1, c2, c3);
         }
       }
-      break;
-    }
-    for (int b = lane; b < 256; b += 32) w.hist[b] = 0u;
-    __syncwarp();
-    for (int base = 0; base < nm; base += 32) {
-      const int i = base + lane;
-      const bool in = i < nm;
-      const int j = in ? (first ? i : w.cand[i]) : 0;
-      hist_add(w.hist, in ? value_bin256(s[j], lo, scale) : 0, in);
-    }
-    __syncwarp();
-    int above, cnt;
-    const int bstar = boundary_bin(w.hist, kk, &above, &cnt);
-    // select the members above the boundary bin; keep its members, in order
-    int nn = 0;
-    float nlo = INFINITY, nhi = -INFINITY;
-    for (int base = 0; base < nm; base += 32) {
-      const int i = base + lane;
-      const bool in = i < nm;
-      const int j = in ? (first ? i : w.cand[i]) : 0;
-      const float x = in ? s[j] : 0.f;
-      const int b = in ? value_bin256(x, lo, scale) : -1;
-      const unsigned keep = __ballot_sync(0xffffffffu, in && b == bstar);  // (reads done)
-      if (first) {
-        const unsigned up = __ballot_sync(0xffffffffu, in && b > bstar);
-        if (lane == 0) w.words[base >> 5] = up;
-      } else if (in && b > bstar) {
-        atomicOr(&w.words[j >> 5], 1u << (j & 31));
+      c1 = static_cast<int>(__reduce_add_sync(0xffffffffu, unsigned(c1)));
+      c2 = static_cast<int>(__reduce_add_sync(0xffffffffu, unsigned(c2)));
+      c3 = static_cast<int>(__reduce_add_sync(0xffffffffu, unsigned(c3)));
+      if (c3 >= k) {
+        tau = t3;
+        cnt = c3;
+      } else if (c2 >= k) {
+        tau = t2;
+        cnt = c2;
+      } else if (c1 >= k) {
+        tau = t1;
+        cnt = c1;
       }
-      if (in && b == bstar) {
-        w.cand[nn + __popc(keep & lanemask_lt())] = j;
-        nlo = fminf(nlo, x);
-        nhi = fmaxf(nhi, x);
-      }
-      nn += __popc(keep);
-      __syncwarp();
     }
+  }
+  // cnt == k: exactly the keys >= tau.  Otherwise tau is the k-th largest
+  // key: every key > tau, then the lowest positions of the keys == tau.
+  const bool exact = cnt == k;
+  // selected outright: keys >= lo (none when tau is the largest key value)
+  const bool none_above = !exact && tau == 0xffffffffu;
+  const uint32_t lo = exact ? tau : tau + 1u;
+  int need = 0;
+  if (none_above) {
+    need = k;
+  } else if (!exact) {
+    int c1 = 0, c2 = 0, c3 = 0;
+    if (compact) {
+      count3(live, lo, lo, lo, c1, c2, c3);
+    } else {
+      count3(key0, lo, lo, lo, c1, c2, c3);
+      for (int c = 1; c < nch; ++c) {
+        uint32_t key[kSelRegs];
+        chunk_keys(sm, n, c, key);
+        count3(key, lo, lo, lo, c1, c2, c3);
+      }
+    }
+    need = k - static_cast<int>(__reduce_add_sync(0xffffffffu, unsigned(c1)));
+  }
+  const uint32_t take_above = none_above ? 0u : 1u;
+  int written = 0;
+  for (int c = 0; c < nch; ++c) {
+    uint32_t key[kSelRegs];
+    if (c == 0) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      nlo = fminf(nlo, __shfl_xor_sync(0xffffffffu, nlo, o));
-      nhi = fmaxf(nhi, __shfl_xor_sync(0xffffffffu, nhi, o));
+      for (int i = 0; i < kSelRegs; ++i) key[i] = key0[i];
+    } else {
+      chunk_keys(sm, n, c, key);
     }
-    kk -= above;
-    nm = nn;
-    lo = nlo;
-    hi = nhi;
-    first = false;
-    __syncwarp();
+    // this lane's selection bits of positions [1024 c + 32 lane, +32)
+    const int base = c * (kSelRegs * 32) + lane * 32;
+    uint32_t word = 0u, ties = 0u;
+#pragma unroll
+    for (int i = 0; i < kSelRegs; ++i) {
+      const int bit = (i + lane) & 31;
+      word |= (uint32_t(key[i] >= lo) & take_above) << bit;
+      ties |= (uint32_t(key[i] == tau) & uint32_t(base + bit < n)) << bit;
+    }
+    if (need > 0) {
+      // the lowest positions of the ties: lanes in order, bits in order
+      const int tc = __popc(ties);
+      int incl = tc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int r = min(max(need - (incl - tc), 0), tc);
+      while (r-- > 0) {
+        word |= ties & (0u - ties);
+        ties &= ties - 1u;
+      }
+      need -= min(need, __shfl_sync(0xffffffffu, incl, 31));
+    }
+    const int wc = __popc(word);
+    int incl = wc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int p = written + incl - wc;
+    while (word) {
+      pos[p++] = base + __ffs(word) - 1;
+      word &= word - 1u;
+    }
+    written += __shfl_sync(0xffffffffu, incl, 31);
   }
   __syncwarp();
-  write_positions(w.words, nw, pos);
 }
 
 // ---------------------------------------------------------------------------
@@ -404,15 +412,13 @@ struct StepSmem {
   static constexpr int RED = up16(kMW * G * (D + 2) * 4);    // warp states
   static constexpr int QF = (D / 16) * 32 * 8;              // Q fragments (one copy)
   static constexpr int QS = D * 4;                           // summed query (fp32)
-  // top-k scratch: hist[256], member positions [nc], selection bits [nc / 32]
-  __host__ __device__ static size_t selw(int nc) { return 256 * 4 + up16(nc * 4) + up16(((nc + 31) / 32) * 4); }
   static constexpr int SELL = (3 * kStepMaxK + 4) * 4;       // positions, prefix, starts
   static constexpr int MISC = kMiscBytes;
   static constexpr int ALIGN = 1024;
   // ring of NS stages, then the rep slice (rep_bytes), the head's scores
   // (nc floats), then the fixed regions
   static size_t bytes(int NS, int rep_bytes, int nc) {
-    return size_t(NS) * Geo::STAGE + up16(rep_bytes) + up16(nc * 4) + RED + QF + QS + selw(nc) +
+    return size_t(NS) * Geo::STAGE + up16(rep_bytes) + up16(nc * 4) + RED + QF + QS +
            SELL + MISC + ALIGN;
   }
 };
@@ -442,8 +448,10 @@ __global__ void __launch_bounds__(kSThreads, 1)
   using S = StepSmem<D, G>;
   constexpr int kSlotF = step_slot_floats(G, D);
   extern __shared__ char smem_raw[];
-  char* ring = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                       ~uintptr_t(1023));
+  // 1024-byte aligned base, offset from the shared array itself (an integer
+  // round trip would hide from the compiler that the pointers address shared
+  // memory and turn every access into a generic one)
+  char* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const AttendArgs& at = a.at;
   const int NS = a.NS;
   const PartOf po = part_of(blockIdx.x, a.P, a.BH);
@@ -459,11 +467,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
   float* red = reinterpret_cast<float*>(reinterpret_cast<char*>(ssc) + S::up16(at.nc * 4));
   uint2* qfrag = reinterpret_cast<uint2*>(reinterpret_cast<char*>(red) + S::RED);
   float* qs = reinterpret_cast<float*>(reinterpret_cast<char*>(qfrag) + S::QF);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(qs) + S::QS);
-  int* cand = reinterpret_cast<int*>(hist + 256);
-  uint32_t* words = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(cand) +
-                                                S::up16(at.nc * 4));
-  int* selpos = reinterpret_cast<int*>(reinterpret_cast<char*>(hist) + S::selw(at.nc));
+  int* selpos = reinterpret_cast<int*>(reinterpret_cast<char*>(qs) + S::QS);
   int* sel_pref = selpos + kStepMaxK;
   int* sel_phys = sel_pref + kStepMaxK + 2;
   const MiscLayout ms(reinterpret_cast<char*>(selpos) + S::SELL);
@@ -538,18 +542,20 @@ __global__ void __launch_bounds__(kSThreads, 1)
       return true;
     };
     // pieces of one kind: rows [v, vend) of the virtual layout given by the
-    // segment prefix `pref` (nseg segments starting at physical rows `phys`),
-    // cut at segment ends and at 64 rows
-    auto run = [&](int v, int vend, const int* pref, const int* phys, int nseg) {
-      const int vlim = min(vend, pref[nseg]);
+    // segment prefix pref(i) (nseg segments starting at physical rows
+    // phys(i)), cut at segment ends and at 64 rows.  (Accessors rather than
+    // arrays: a small array indexed at run time would live in local memory,
+    // and every access to it would wait on an L2 kept busy by the copies.)
+    auto run = [&](int v, int vend, auto pref, auto phys, int nseg) {
+      const int vlim = min(vend, pref(nseg));
       while (alive && v < vlim) {
         int lo2 = 0, hi2 = nseg - 1;
         while (lo2 < hi2) {
           const int mid = (lo2 + hi2 + 1) >> 1;
-          if (pref[mid] <= v) lo2 = mid; else hi2 = mid - 1;
+          if (pref(mid) <= v) lo2 = mid; else hi2 = mid - 1;
         }
-        const int n = min(min(vlim, pref[lo2 + 1]), v + kMTT) - v;
-        const int y = static_cast<int>(int64_t(bh) * at.cap + phys[lo2] + (v - pref[lo2]));
+        const int n = min(min(vlim, pref(lo2 + 1)), v + kMTT) - v;
+        const int y = static_cast<int>(int64_t(bh) * at.cap + phys(lo2) + (v - pref(lo2)));
         if (pend && !emit(pn, py, false)) {
           alive = false;
           break;
@@ -561,9 +567,10 @@ __global__ void __launch_bounds__(kSThreads, 1)
       }
     };
     {
-      const int st_pref[3] = {0, at.sink_end, a.L_st};
-      const int st_phys[2] = {0, static_cast<int>(at.w0)};
-      run(xs0, xs1, st_pref, st_phys, 2);
+      // sink rows [0, sink_end) then window rows [w0, T): two segments
+      const int se = at.sink_end, lst = a.L_st, w0 = static_cast<int>(at.w0);
+      run(xs0, xs1, [=](int i) { return i == 0 ? 0 : (i == 1 ? se : lst); },
+          [=](int i) { return i == 0 ? 0 : w0; }, 2);
     }
     if (alive) {
       // the selector fills sel_pref / sel_phys and arrives on sel (also
@@ -574,7 +581,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
           *ms.abort_flag != 0)
         alive = false;
       else if (xq1 > xq0)
-        run(xq0, xq1, sel_pref, sel_phys, at.k);
+        run(xq0, xq1, [=](int i) { return sel_pref[i]; }, [=](int i) { return sel_phys[i]; }, at.k);
     }
     if (alive) emit(pend ? pn : 0, py, true);
     // no copy may still be landing in shared memory when the CTA exits
@@ -609,23 +616,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok) {
-      // eight loads in flight per lane before any store (a store through a
-      // generic pointer would otherwise order every next load after it)
-      const float* src = a.scores + int64_t(bh) * at.nc;
-      for (int base = 0; base < at.nc; base += 256) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int jj = base + u * 32 + lane;
-          v[u] = jj < at.nc ? ld_cg_f32(src + jj) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (base + u * 32 + lane < at.nc) ssc[base + u * 32 + lane] = v[u];
-      }
-      __syncwarp();
-      const WarpTopkSmem wt{hist, cand, words};
-      warp_topk(ssc, at.nc, at.k, selpos, wt);
+      // (live-key scratch: selpos and the start of sel_pref, both written after it)
+      warp_topk(a.scores + int64_t(bh) * at.nc, ssc, reinterpret_cast<uint32_t*>(selpos), at.nc,
+                at.k, selpos);
       // the selected blocks as segments of the attended set (clipped to
       // [sink, w0)), prefix of their lengths; part 0 writes the selection out
       int run = 0;
@@ -904,6 +897,7 @@ bool step_plan(const rba_store* st, const Geometry& g, StepPlan* pl) {
 
 bool step_eligible(const rba_store* st, const Geometry& g, int k) {
   const rba_store_desc& d = st->d;
+  if (st->one_launch == 0) return false;
   if (d.dtype != RBA_BF16 || (st->pitch != 64 && st->pitch != 128)) return false;
   if (d.block_size % kMTT != 0) return false;
   if (d.mode != RBA_REP_MEAN && d.mode != RBA_REP_TOPR_ATTN && d.mode != RBA_REP_EXTERNAL)

@@ -312,7 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap map_ck,
                    const __grid_constant__ CUtensorMap map_cv) {
   extern __shared__ char smem_raw[];
-  char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, offset from the shared array itself (an integer
+  // round trip would hide from the compiler that the pointers address shared
+  // memory and turn every access into a generic one)
+  char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   char* sQ = smem + kQOff;
   int4* tiles = reinterpret_cast<int4*>(smem + kTileOff);
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);

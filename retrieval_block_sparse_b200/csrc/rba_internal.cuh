@@ -20,6 +20,7 @@ struct rba_store {
   int64_t cap_blocks;
   int32_t score_reduce;   // rba_score_reduce: how a block's r representative keys combine
   unsigned long long wait_ns;  // bound of the one-launch decode step's waits (ns)
+  int32_t one_launch;     // rba_decode_step may use the one-launch path (0: three kernels)
 };
 
 namespace rba {
@@ -91,10 +92,13 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 // ---------------------------------------------------------------------------
 // top-k keys: larger key = better (higher score, then lower position)
 
+// (straight-line arithmetic: a branch on the loaded value would make every
+// load in an unrolled loop complete before the next one issues)
 __device__ __forceinline__ uint32_t ordered_f32(float f) {
   uint32_t u = __float_as_uint(f);
-  if ((u << 1) == 0) u = 0;  // -0 == +0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  u &= 0u - uint32_t((u << 1) != 0u);  // -0 == +0
+  const uint32_t flip = uint32_t(int32_t(u) >> 31) | 0x80000000u;  // negative: all bits
+  return u ^ flip;
 }
 __device__ __forceinline__ uint64_t topk_key(float s, uint32_t pos) {
   return (static_cast<uint64_t>(ordered_f32(s)) << 32) | static_cast<uint32_t>(0xffffffffu - pos);

@@ -146,6 +146,7 @@ rba_status rba_store_create(const rba_store_desc* d, void* k_pool, void* v_pool,
   s->cap_blocks = d->capacity_tokens / d->block_size;
   s->score_reduce = RBA_SCORE_SUM;
   s->wait_ns = rba::kDefaultWaitNs;
+  s->one_launch = 0;
   *out = s;
   return RBA_OK;
 }
@@ -201,6 +202,12 @@ int32_t rba_version(void) { return 100; }
 extern "C" rba_status rba_store_set_wait_limit_ns(rba_store* st, uint64_t ns) {
   if (st == nullptr) return RBA_ERR_INVALID_ARG;
   st->wait_ns = ns == 0 ? rba::kDefaultWaitNs : ns;
+  return RBA_OK;
+}
+
+extern "C" rba_status rba_store_set_decode_step_one_launch(rba_store* st, int32_t on) {
+  if (st == nullptr || (on != 0 && on != 1)) return RBA_ERR_INVALID_ARG;
+  st->one_launch = on;
   return RBA_OK;
 }
 

@@ -29,6 +29,7 @@ SIGNATURES = {
     "rba_store_destroy": (_c_i32, [_p]),
     "rba_store_set_score_reduce": (_c_i32, [_p, _c_i32]),
     "rba_store_set_wait_limit_ns": (_c_i32, [_p, ctypes.c_uint64]),
+    "rba_store_set_decode_step_one_launch": (_c_i32, [_p, _c_i32]),
     "rba_candidates": (_c_i32, [_p, _c_i64, _c_i32, _c_i32, ctypes.POINTER(_c_i32),
                                 ctypes.POINTER(_c_i32)]),
     "rba_memorize": (_c_i32, [_p, _p, _p, _c_i64, _c_i32, _p, _c_i32, _c_f32, _p]),
@@ -196,6 +197,11 @@ class Store:
         """Bound of the one-launch decode step's device waits (0: the default 2 s)."""
         _check(lib().rba_store_set_wait_limit_ns(self.handle, int(ns)),
                "rba_store_set_wait_limit_ns")
+
+    def set_decode_step_one_launch(self, on=True):
+        """Let decode_step run as one cooperative launch where eligible (plan 3)."""
+        _check(lib().rba_store_set_decode_step_one_launch(self.handle, int(bool(on))),
+               "rba_store_set_decode_step_one_launch")
 
     def __del__(self):
         h = getattr(self, "handle", None)

@@ -38,11 +38,14 @@ def host_bits(t, dtype):
     return t.detach().cpu().numpy()
 
 
-def make_decode_store(rba, w, x):
-    """Store holding the whole context of workload w, representations memorised."""
+def make_decode_store(rba, w, x, one_launch=False):
+    """Store holding the whole context of workload w, representations memorised;
+    one_launch lets its decode step run as one cooperative launch."""
     st = rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                    head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
                    dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep)
+    if one_launch:
+        st.set_decode_step_one_launch(True)
     st.kv_rows(st.k).copy_(dev(x["K"], w.dtype))  # (pool rows may be padded past D)
     st.kv_rows(st.v).copy_(dev(x["V"], w.dtype))
     aux = None

@@ -126,10 +126,11 @@ def test_attend_on_oracle_selection(rba, name):
     np.testing.assert_allclose(lse, ref["lse"], rtol=0, atol=OUT_TOL[w.dtype])
 
 
+@pytest.mark.parametrize("one_launch", [False, True])
 @pytest.mark.parametrize("name", NAMES)
-def test_decode_step(rba, name):
+def test_decode_step(rba, name, one_launch):
     w, x, reps, pos, ref = _prepared(name)
-    st = make_decode_store(rba, w, x)
+    st = make_decode_store(rba, w, x, one_launch)
     q = dev(x["q"], w.dtype)
     ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)
     for _ in range(2):  # the workspace must be reusable call after call

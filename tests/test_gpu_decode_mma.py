@@ -54,8 +54,8 @@ def _prepared(name):
 def test_attend_on_oracle_selection(rba, name):
     w, x, ref = _prepared(name)
     st = make_decode_store(rba, w, x)
-    # rba_attend runs the whole-block kernel (the decode step may run in one launch)
-    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) in (2, 3)
+    # rba_attend runs the whole-block kernel, as the default decode step does
+    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 2
     idx = torch.from_numpy(ref["idx"].astype(np.int32)).cuda()
     out, lse = st.attend(dev(x["q"], w.dtype), idx, w.context, w.sink, w.window)
     st.check()
@@ -71,10 +71,16 @@ def test_attend_on_oracle_selection(rba, name):
     np.testing.assert_allclose(lse, ref["lse"], rtol=0, atol=OUT_TOL[w.dtype])
 
 
+@pytest.mark.parametrize("one_launch", [False, True])
 @pytest.mark.parametrize("name", list(CASES))
-def test_decode_step(rba, name):
+def test_decode_step(rba, name, one_launch):
     w, x, ref = _prepared(name)
-    st = make_decode_store(rba, w, x)
+    st = make_decode_store(rba, w, x, one_launch)
+    # 8 x 32 (batch, kv head) units are more than the one launch takes (at most
+    # half as many as SMs): that case keeps the three-kernel step
+    one = one_launch and w.batch * w.n_kv_heads * 2 <= torch.cuda.get_device_properties(
+        0).multi_processor_count
+    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == (3 if one else 2)
     q = dev(x["q"], w.dtype)
     ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)
     for _ in range(2):  # the workspace is reusable call after call

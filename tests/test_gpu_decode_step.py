@@ -1,13 +1,15 @@
-"""GPU parity of the one-launch decode step (rba_decode_step where
-rba_decode_step_plan() reports 3) against the fp64 oracle, through the C ABI.
+"""GPU parity of the one-launch decode step (rba_decode_step on a store with
+rba_store_set_decode_step_one_launch(store, 1), where rba_decode_step_plan()
+reports 3) against the fp64 oracle, through the C ABI.
 
-The whole-step tests of test_gpu_decode.py, test_gpu_decode_mma.py and
-test_gpu_score_max.py already run this kernel on the configurations it covers
+The whole-step tests of test_gpu_decode.py, test_gpu_decode_mma.py,
+test_gpu_fused.py and test_gpu_score_max.py run this kernel and the default
+three-kernel step on the configurations they cover
 (GQA 1, 2 and 4, head dims 64 and 128, mean / top-r representations with 1, 2,
 4 and 8 keys, sum and max scores).  This file adds what those random inputs do
 not reach: exact score ties at the k-th place (the lower block index must win,
-as in the oracle), a row of equal scores and a row whose k-th score sits in a
-crowded value bin (both take the selector's exact radix path), a part count
+as in the oracle), a row of equal scores and a row whose k-th score sits
+among many near-equal scores (long radix searches), a part count
 that leaves some parts without candidates, and the bounded waits: with a wait
 limit of 1 ns the step must report RBA_ERR_TIMEOUT in the status word and
 return, and the next call on the same workspace must match the oracle."""
@@ -28,7 +30,7 @@ SMALL = BASE.scaled(context=16384, window=1024, top_k=16, n_planted=8, seed=61)
 def _run_with_reps(rba, w, x, reps):
     """Store with the given representations written into its rep pool, one
     decode step, and the oracle on the same representations."""
-    st = make_decode_store(rba, w, x)
+    st = make_decode_store(rba, w, x, one_launch=True)
     assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 3
     rb = torch.from_numpy(reps.astype(np.float32)).to(torch.bfloat16)
     st.rep.copy_(rb.cuda())
@@ -41,15 +43,21 @@ def _run_with_reps(rba, w, x, reps):
     return st, ref, idx.cpu().numpy(), out.cpu().numpy(), lse.cpu().numpy()
 
 
-def test_plan_is_one_launch_at_128k(rba):
+def test_plan_at_128k(rba):
     w = BASE
     x = synth.decode_inputs(w.scaled(context=8192, window=1024, n_planted=4))
     st = rba.Store(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                    head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
                    dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep)
     del x
+    # the three-kernel step by default; one launch when asked for
+    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 2
+    assert st.decode_launches(w.top_k, w.context, w.sink, w.window) == 3
+    st.set_decode_step_one_launch(True)
     assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 3
     assert st.decode_launches(w.top_k, w.context, w.sink, w.window) == 1
+    st.set_decode_step_one_launch(False)
+    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 2
 
 
 def test_exact_ties_take_the_lower_block(rba):
@@ -90,9 +98,10 @@ def test_equal_scores_select_the_first_candidates(rba):
 
 
 def test_crowded_boundary_bin(rba):
-    # two far outliers stretch the value range, so the remaining scores all
-    # fall into a few of the 256 value bins: more than 32 members share the
-    # bin of the k-th score and the selector ranks them exactly (radix path)
+    # two far outliers stretch the value range while the remaining scores
+    # crowd near one value: the k-th score shares its high bits with most of
+    # the row, so the radix search runs down to the low bits (and a binning
+    # select would hold them in one bin)
     w = SMALL
     x = synth.decode_inputs(w)
     reps, _ = oracle_reps(w, x)
@@ -118,7 +127,7 @@ def test_parts_without_candidates(rba):
                     n_planted=2, seed=63)
     x = synth.decode_inputs(w)
     reps, _ = oracle_reps(w, x)
-    st = make_decode_store(rba, w, x)
+    st = make_decode_store(rba, w, x, one_launch=True)
     assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 3
     ref = O.decode(x["q"], x["K"], x["V"], reps, dtype=w.dtype, block_size=w.block_size,
                    sink=w.sink, window=w.window, top_k_blocks=w.top_k)
@@ -135,7 +144,7 @@ def test_wait_that_runs_out_reports_timeout_and_next_call_is_correct(rba):
     w = SMALL
     x = synth.decode_inputs(w)
     reps, _ = oracle_reps(w, x)
-    st = make_decode_store(rba, w, x)
+    st = make_decode_store(rba, w, x, one_launch=True)
     assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 3
     q = dev(x["q"], w.dtype)
     ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)

@@ -32,11 +32,12 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("one_launch", [False, True])
 @pytest.mark.parametrize("name", list(CASES))
-def test_fused_step_equals_three_launches(rba, name):
+def test_fused_step_equals_three_launches(rba, name, one_launch):
     w = CASES[name]
     x = synth.decode_inputs(w)
-    st = make_decode_store(rba, w, x)
+    st = make_decode_store(rba, w, x, one_launch)
     q = dev(x["q"], w.dtype)
     first, nc = st.candidates(w.context, w.sink, w.window)
     scores = st.score(q, w.context, w.sink, w.window)
@@ -44,13 +45,13 @@ def test_fused_step_equals_three_launches(rba, name):
         w.batch, w.n_kv_heads, w.top_k)
     out3, lse3 = st.attend(q, idx3, w.context, w.sink, w.window)
     plan = st.decode_plan(w.top_k, w.context, w.sink, w.window)
-    # bf16 always takes a persistent kernel: the one-launch step (plan 3) or
-    # the whole-block tensor-core attention kernel (plan 2) when blocks are
-    # whole 64-row tiles; fp32 with one q head per kv head has tiles too large
-    # for shared memory and runs split-K (plan -2)
+    # bf16 always takes a persistent kernel: the one-launch step (plan 3, when
+    # asked for) or the whole-block tensor-core attention kernel (plan 2) when
+    # blocks are whole 64-row tiles; fp32 with one q head per kv head has
+    # tiles too large for shared memory and runs split-K (plan -2)
     whole = w.block_size % 64 == 0
     if w.dtype == "bf16":
-        assert plan in ((2, 3) if whole else (1,)), plan
+        assert plan == ((3 if one_launch else 2) if whole else 1), plan
     else:
         assert plan in (1, -2), plan
     ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)

@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 W = synth.WORKLOADS
 D = 100
 DECODE = {
-    # one launch: 32 MHA heads of 100 (B = 1), top-r representative keys
+    # one launch (asked for): 32 MHA heads of 100 (B = 1), top-r representative keys
     "step-mha32": (W["infllm-decode-128k"].scaled(n_q_heads=32, n_kv_heads=32, head_dim=D,
                                                   context=16384, window=1024, top_k=16,
                                                   n_planted=8, seed=81), 3),
@@ -45,7 +45,7 @@ def test_decode_step_d100(rba, name):
     w, plan = DECODE[name]
     x = synth.decode_inputs(w)
     reps, pos = oracle_reps(w, x)
-    st = make_decode_store(rba, w, x)
+    st = make_decode_store(rba, w, x, one_launch=plan == 3)
     assert st.pitch == 128 and st.k.shape[-1] == 128
     if plan is not None:
         assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == plan

@@ -39,14 +39,17 @@ def _store(rba, w, x):
     return st
 
 
+@pytest.mark.parametrize("one_launch", [False, True])
 @pytest.mark.parametrize("name", list(CASES))
-def test_max_scores_and_decode_step(rba, name):
+def test_max_scores_and_decode_step(rba, name, one_launch):
     w = CASES[name]
     x = synth.decode_inputs(w)
     reps, _ = oracle_reps(w, x)
     ref = O.decode(x["q"], x["K"], x["V"], reps, dtype=w.dtype, block_size=w.block_size,
                    sink=w.sink, window=w.window, top_k_blocks=w.top_k, score_reduce="max")
     st = _store(rba, w, x)
+    if one_launch:
+        st.set_decode_step_one_launch(True)
     q = dev(x["q"], w.dtype)
     s = st.score(q, w.context, w.sink, w.window).cpu().numpy().astype(np.float64)
     st.check()
