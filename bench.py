@@ -679,6 +679,7 @@ def measure_decode_config(name, dev, seconds, pk, score_reduce="sum", workload=N
                      2: "pipelined, persistent attention (whole-block, tensor cores)",
                      3: "one cooperative launch (score, top-k, tensor-core attention)"}.get(
                          plan, "split-K attention"),
+            "kernels_per_step": st.decode_launches(w.top_k, w.context, w.sink, w.window),
             "steps_timed": n * len(stores),
             "l2": (f"L2-sized write between steps, its time subtracted" if use_flush else
                    f"{len(stores)} store replicas rotated ({len(stores)} x {nbytes / 1e6:.1f} MB"

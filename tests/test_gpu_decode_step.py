@@ -1,6 +1,8 @@
-"""GPU parity of the one-launch decode step (rba_decode_step on a store with
-rba_store_set_decode_step_one_launch(store, 1), where rba_decode_step_plan()
-reports 3) against the fp64 oracle, through the C ABI.
+"""GPU parity of the decode step's selection paths against the fp64 oracle,
+through the C ABI: the one-launch step (rba_decode_step on a store with
+rba_store_set_decode_step_one_launch(store, 1), plan 3; one selecting warp
+per part) and, on the same tie cases, the default score -> top-k ->
+attention step (rba_topk's kernel).
 
 The whole-step tests of test_gpu_decode.py, test_gpu_decode_mma.py,
 test_gpu_fused.py and test_gpu_score_max.py run this kernel and the default
@@ -27,11 +29,13 @@ BASE = synth.WORKLOADS["infllm-decode-128k"]
 SMALL = BASE.scaled(context=16384, window=1024, top_k=16, n_planted=8, seed=61)
 
 
-def _run_with_reps(rba, w, x, reps):
+def _run_with_reps(rba, w, x, reps, one_launch):
     """Store with the given representations written into its rep pool, one
-    decode step, and the oracle on the same representations."""
-    st = make_decode_store(rba, w, x, one_launch=True)
-    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 3
+    decode step (one launch, or the default score -> top-k -> attention), and
+    the oracle on the same representations."""
+    st = make_decode_store(rba, w, x, one_launch=one_launch)
+    assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == (3 if one_launch else 2)
+    assert st.decode_launches(w.top_k, w.context, w.sink, w.window) == (1 if one_launch else 3)
     rb = torch.from_numpy(reps.astype(np.float32)).to(torch.bfloat16)
     st.rep.copy_(rb.cuda())
     reps_stored = rb.float().numpy().astype(np.float64)  # the values the GPU reads
@@ -50,7 +54,8 @@ def test_plan_at_128k(rba):
                    head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
                    dtype=w.dtype, mode=w.rep_mode, n_rep=w.n_rep)
     del x
-    # the three-kernel step by default; one launch when asked for
+    # by default score -> top-k -> whole-block attention; one launch when
+    # asked for
     assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 2
     assert st.decode_launches(w.top_k, w.context, w.sink, w.window) == 3
     st.set_decode_step_one_launch(True)
@@ -60,7 +65,8 @@ def test_plan_at_128k(rba):
     assert st.decode_plan(w.top_k, w.context, w.sink, w.window) == 2
 
 
-def test_exact_ties_take_the_lower_block(rba):
+@pytest.mark.parametrize("one_launch", [True, False])
+def test_exact_ties_take_the_lower_block(rba, one_launch):
     # copy the representation of the oracle's k-th block onto candidates just
     # below and just above it in index: their scores equal the k-th exactly,
     # so the lower index must be selected, bit for bit as in the oracle
@@ -78,26 +84,28 @@ def test_exact_ties_take_the_lower_block(rba):
         for j in (kth - 3, kth + 5):  # neighbours outside the selection
             if cand[0] <= j < cand[0] + cand.size and j not in ref["idx"][0, h]:
                 reps[0, h, j] = reps[0, h, kth]
-    st, ref2, idx, out, lse = _run_with_reps(rba, w, x, reps)
+    st, ref2, idx, out, lse = _run_with_reps(rba, w, x, reps, one_launch)
     np.testing.assert_array_equal(idx, ref2["idx"])
     check_decode_step(w, x["q"], x["K"], x["V"], ref2, idx, out, lse, min_exact=1.0)
 
 
-def test_equal_scores_select_the_first_candidates(rba):
+@pytest.mark.parametrize("one_launch", [True, False])
+def test_equal_scores_select_the_first_candidates(rba, one_launch):
     # every block represented by the same keys: one score per head, a zero
     # value range; the k lowest candidate blocks are selected
     w = SMALL
     x = synth.decode_inputs(w)
     reps, _ = oracle_reps(w, x)
     reps[:] = reps[:, :, :1]
-    st, ref, idx, out, lse = _run_with_reps(rba, w, x, reps)
+    st, ref, idx, out, lse = _run_with_reps(rba, w, x, reps, one_launch)
     first = int(ref["cand"][0])
     np.testing.assert_array_equal(idx, np.broadcast_to(np.arange(first, first + w.top_k),
                                                        idx.shape))
     check_decode_step(w, x["q"], x["K"], x["V"], ref, idx, out, lse, min_exact=1.0)
 
 
-def test_crowded_boundary_bin(rba):
+@pytest.mark.parametrize("one_launch", [True, False])
+def test_crowded_boundary_bin(rba, one_launch):
     # two far outliers stretch the value range while the remaining scores
     # crowd near one value: the k-th score shares its high bits with most of
     # the row, so the radix search runs down to the low bits (and a binning
@@ -115,7 +123,7 @@ def test_crowded_boundary_bin(rba):
         u = qs / np.linalg.norm(qs)
         reps[0, h, 10] = base[0, h, 0] + 400.0 * u / w.n_rep   # far above
         reps[0, h, 20] = base[0, h, 0] - 400.0 * u / w.n_rep   # far below
-    st, ref, idx, out, lse = _run_with_reps(rba, w, x, reps)
+    st, ref, idx, out, lse = _run_with_reps(rba, w, x, reps, one_launch)
     check_decode_step(w, x["q"], x["K"], x["V"], ref, idx, out, lse)
     assert all(10 in idx[0, h] and 20 not in idx[0, h] for h in range(w.n_kv_heads))
 
