@@ -971,29 +971,27 @@ struct FusedKernel {
   }
 };
 
-// CTAs of this kernel that fit on one SM (0: none; <0: a CUDA error)
+// CTAs of this kernel that fit on one SM (0: none; <0: a CUDA error); the
+// query is cached per device (every decode step asks)
 template <typename T, int D, int G, bool MMA>
 int fused_occupancy_t() {
   using K = FusedKernel<T, D, G, MMA>;
   const size_t smem = K::smem(K::stages());
   if (smem > kMaxSmem) return 0;  // (large fp32 tiles) the split-K kernel runs instead
-  if (ensure_smem(K::fn(), smem) != cudaSuccess) return -1;
-  int occ = 0;
-  const cudaError_t e =
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, K::fn(), K::kThreads, smem);
-  if (getenv("RBA_DEBUG") != nullptr) {
-    cudaFuncAttributes fa = {};
-    cudaFuncGetAttributes(&fa, K::fn());
-    fprintf(stderr,
-            "rba: decode attention kernel (%s) regs=%d maxThreads=%d static_smem=%zu local=%zu "
-            "max_dyn_smem=%d requested_smem=%zu threads=%d occupancy=%d (%s)\n",
-            MMA ? "tensor-core, whole blocks" : "cuda-core", fa.numRegs, fa.maxThreadsPerBlock,
-            fa.sharedSizeBytes, fa.localSizeBytes, fa.maxDynamicSharedSizeBytes, smem,
-            K::kThreads, occ, cudaGetErrorString(e));
-  }
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return -2;
+  const int occ = occupancy(K::fn(), K::kThreads, smem);
+  static const bool debug = getenv("RBA_DEBUG") != nullptr;
+  if (debug) {
+    static std::once_flag once;
+    std::call_once(once, [&] {
+      cudaFuncAttributes fa = {};
+      cudaFuncGetAttributes(&fa, K::fn());
+      fprintf(stderr,
+              "rba: decode attention kernel (%s) regs=%d maxThreads=%d static_smem=%zu "
+              "local=%zu max_dyn_smem=%d requested_smem=%zu threads=%d occupancy=%d\n",
+              MMA ? "tensor-core, whole blocks" : "cuda-core", fa.numRegs, fa.maxThreadsPerBlock,
+              fa.sharedSizeBytes, fa.localSizeBytes, fa.maxDynamicSharedSizeBytes, smem,
+              K::kThreads, occ);
+    });
   }
   return occ;
 }
@@ -1189,12 +1187,8 @@ rba_status launch_fused(const rba_store* st, const void* q, int k, const Geometr
     a.ps[c] = static_cast<int>(xs);
   }
   CUtensorMap maps[2];
-  if (mma) {
-    const int64_t rows = int64_t(d.batch) * d.n_kv_heads * d.capacity_tokens;
-    if (!make_tmap_bf16(&maps[0], st->k, rows, st->pitch, kMTT) ||
-        !make_tmap_bf16(&maps[1], st->v, rows, st->pitch, kMTT))
-      return RBA_ERR_CUDA;
-  }
+  static_assert(kMTT == 64, "the store's cached tensor maps use 64-row boxes");
+  if (mma && !store_tmaps64(st, &maps[0], &maps[1])) return RBA_ERR_CUDA;
   const int G = d.n_q_heads / d.n_kv_heads;
 #define RBA_FUSED(T_, D_, M_)                                                   \
   switch (G) {                                                                  \

@@ -969,10 +969,8 @@ rba_status launch_step(const rba_store* st, const void* q, int k, const Geometry
   a.max_over_keys = st->score_reduce == RBA_SCORE_MAX ? 1 : 0;
   a.wait_ns = st->wait_ns;
   CUtensorMap maps[2];
-  const int64_t rows = int64_t(d.batch) * d.n_kv_heads * d.capacity_tokens;
-  if (!make_tmap_bf16(&maps[0], st->k, rows, st->pitch, kMTT) ||
-      !make_tmap_bf16(&maps[1], st->v, rows, st->pitch, kMTT))
-    return RBA_ERR_CUDA;
+  static_assert(kMTT == 64, "the store's cached tensor maps use 64-row boxes");
+  if (!store_tmaps64(st, &maps[0], &maps[1])) return RBA_ERR_CUDA;
   const void* fn = step_kernel(st);
   if (fn == nullptr) return RBA_ERR_UNSUPPORTED;
   RBA_CUDA_TRY(ensure_smem(fn, pl.smem));

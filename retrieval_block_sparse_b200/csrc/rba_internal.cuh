@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include <cuda.h>
 
 #include "rba.h"
@@ -21,6 +23,11 @@ struct rba_store {
   int32_t score_reduce;   // rba_score_reduce: how a block's r representative keys combine
   unsigned long long wait_ns;  // bound of the one-launch decode step's waits (ns)
   int32_t one_launch;     // rba_decode_step may use the one-launch path (0: three kernels)
+  // tensor maps of the K and V pools in 64-row boxes (the whole-block decode
+  // kernels), encoded once on first use: the pools never move
+  mutable std::once_flag tmap_once;
+  mutable bool tmap_ok = false;
+  mutable CUtensorMap kmap64 = {}, vmap64 = {};
 };
 
 namespace rba {
@@ -167,6 +174,9 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // zero fill outside the matrix.  False if the driver's encoder is unavailable
 // or rejects the arguments.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int cols, int box_rows);
+// the store's K and V tensor maps in 64-row boxes (encoded once); false if
+// they cannot be encoded
+bool store_tmaps64(const rba_store* st, CUtensorMap* kmap, CUtensorMap* vmap);
 inline size_t dtype_size(rba_dtype t) { return t == RBA_BF16 ? 2 : 4; }
 // Row pitch (elements) of the pools for a head dim: 64 up to 64, else 128;
 // -1 for head dims the library does not hold (not a multiple of 4, or > 128).

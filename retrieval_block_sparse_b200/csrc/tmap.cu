@@ -43,4 +43,16 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int cols, in
          CUDA_SUCCESS;
 }
 
+bool store_tmaps64(const rba_store* st, CUtensorMap* kmap, CUtensorMap* vmap) {
+  std::call_once(st->tmap_once, [st] {
+    const int64_t rows = int64_t(st->d.batch) * st->d.n_kv_heads * st->d.capacity_tokens;
+    st->tmap_ok = make_tmap_bf16(&st->kmap64, st->k, rows, st->pitch, 64) &&
+                  make_tmap_bf16(&st->vmap64, st->v, rows, st->pitch, 64);
+  });
+  if (!st->tmap_ok) return false;
+  *kmap = st->kmap64;
+  *vmap = st->vmap64;
+  return true;
+}
+
 }  // namespace rba
