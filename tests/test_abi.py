@@ -183,3 +183,20 @@ def test_score_reduce_setter_checks(L):
     assert L.rba_store_set_score_reduce(h, 1) == 1
     L.rba_store_destroy(h)
     assert L.rba_store_set_score_reduce(None, 1) == 1
+
+
+def test_step_setters_check_their_arguments(L):
+    # the one-launch switch takes 0 or 1; the wait bound takes any value (0:
+    # the default); both reject a NULL store.  Host only: nothing launches.
+    L.rba_store_set_decode_step_one_launch.argtypes = [ctypes.c_void_p, ctypes.c_int32]
+    L.rba_store_set_wait_limit_ns.argtypes = [ctypes.c_void_p, ctypes.c_uint64]
+    s, h = _create(L)
+    assert L.rba_store_set_decode_step_one_launch(h, 1) == 0
+    assert L.rba_store_set_decode_step_one_launch(h, 0) == 0
+    assert L.rba_store_set_decode_step_one_launch(h, 2) == 1
+    assert L.rba_store_set_decode_step_one_launch(h, -1) == 1
+    assert L.rba_store_set_wait_limit_ns(h, 0) == 0
+    assert L.rba_store_set_wait_limit_ns(h, 1000) == 0
+    L.rba_store_destroy(h)
+    assert L.rba_store_set_decode_step_one_launch(None, 1) == 1
+    assert L.rba_store_set_wait_limit_ns(None, 0) == 1
