@@ -509,10 +509,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_us / 1e3, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generator; K,V~N(0,1), planted per-head bias, 16-query probe)",
-        "config": {"workload": args.workload, "batch": w.batch, "q_heads": w.n_q_heads,
-                   "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context": w.context,
-                   "block_size": w.block_size, "rep_keys": w.n_rep, "top_k": w.top_k,
-                   "sink": w.sink, "window": w.window, "candidates": nc,
+        "config": {**workload_config(args.workload, w, nc),
                    "l2": f"inputs larger than L2: {R} store replicas rotated "
                          f"({R} x {bytes_step / 1e6:.1f} MB >= 4 x {l2 / 1e6:.0f} MB L2)",
                    "parallelism": f"replicas x{world} (no exchange step)",
@@ -1033,6 +1030,14 @@ def cpu_baseline(w, x, seconds, workload=WORKLOAD):
                       f"cores = BLAS threads used"}
 
 
+def workload_config(name, w, nc):
+    """The workload part of a bench line's config (the same in both arms)."""
+    return {"workload": name, "batch": w.batch, "q_heads": w.n_q_heads,
+            "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context": w.context,
+            "block_size": w.block_size, "rep_keys": w.n_rep, "top_k": w.top_k,
+            "sink": w.sink, "window": w.window, "candidates": nc}
+
+
 def run_reference(args):
     """The oracle as the reference arm: each reference step is a bounded sample
     of whole decode steps (every (batch, kv head) unit of the workload), sized
@@ -1042,8 +1047,10 @@ def run_reference(args):
     if rank != 0:
         return None
     from retrieval_block_sparse_b200 import synth
+    import oracle as O
     w = synth.WORKLOADS[args.workload]
     x = synth.decode_inputs(w)
+    nc = int(O.candidate_blocks(w.context, w.block_size, w.sink, w.window).size)
     unit, per_step = _oracle_units(w, x)
     t0 = time.perf_counter()
     n_warm = max(args.warmup, 1) * per_step
@@ -1077,7 +1084,7 @@ def run_reference(args):
             "ms_per_step": round(el * 1e3 / n_dec, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded generator)", "impl": "reference",
-            "config": {"workload": args.workload},
+            "config": workload_config(args.workload, w, nc),
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores,
                              "kind": "oracle", "sample": desc, **_host_cpu()},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
