@@ -323,9 +323,10 @@ size_t rba_decode_step_workspace_size(const rba_store* store, int32_t k, int64_t
  *   2   score -> top-k -> persistent attention kernel, the last two as programmatic
  *       dependents (overlapped); the attention kernel is the whole-block one: bf16 store,
  *       block size a multiple of 64, head dim 64 or 128; inner products on tensor cores
- *   1   as 2 with the CUDA-core attention kernel (other block sizes, fp32); k <= 2048,
- *       GQA group of 1, 2 or 4 in both
- *   0   score -> top-k -> split-K attention, in stream order: outside those limits
+ *   1   as 2 with the CUDA-core attention kernel (other block sizes of at least 2, fp32);
+ *       k <= 2048, GQA group of 1, 2 or 4 in both
+ *   0   score -> top-k -> split-K attention, in stream order: outside those limits, and
+ *       token-level stores (block size 1, where gathered loads beat per-row bulk copies)
  *  -2   within the limits but no CTA of the persistent kernel fits on an SM (as 0)
  *  -3   a CUDA error while asking (as 0)
  *  -4   invalid arguments (as rba_decode_step would report) */
@@ -334,7 +335,7 @@ int32_t rba_decode_step_plan(const rba_store* store, int32_t k, int64_t T, int32
 
 /* Number of kernels rba_decode_step enqueues for this problem (host only, launches
  * nothing): 1 where rba_decode_step_plan() reports 3; else block scores and top-k (one
- * kernel for rows of up to 8192 candidates, four above; neither when k = 0), then one
+ * kernel for rows of up to 16384 candidates, four above; neither when k = 0), then one
  * attention kernel (persistent or split-K).  -4 for invalid arguments. */
 int32_t rba_decode_step_launches(const rba_store* store, int32_t k, int64_t T, int32_t sink,
                                  int32_t window);

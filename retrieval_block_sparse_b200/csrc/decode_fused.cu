@@ -1093,8 +1093,14 @@ size_t fused_sync_bytes(const rba_store* st) {
 
 // Whether the persistent attention kernel covers this problem (else the
 // split-K kernel runs).
+// Token-level retrieval (one key per block) runs split-K: the persistent
+// kernels stage each selected row with its own bulk copies, and the split-K
+// kernel's gathered 16-byte loads cost less (1M-token decode 528 -> 508 us,
+// two-stage retrieval 108 -> 91 us per step on B200).
+constexpr int kFusedMinBlock = 2;
 bool fused_eligible(const rba_store* st, const Geometry& g, int k) {
   const rba_store_desc& d = st->d;
+  if (d.block_size < kFusedMinBlock) return false;
   const int G = d.n_q_heads / d.n_kv_heads;
   if (d.mode == RBA_REP_EMBED_COSINE) return false;
   if (G != 1 && G != 2 && G != 4) return false;

@@ -5,8 +5,9 @@
 
 namespace rba {
 
-// Rows of at most kSmallN scores are selected by one CTA in shared memory.
-constexpr int kSmallN = 8192;
+// Rows of at most kSmallN scores are selected by one CTA in shared memory
+// (5 bytes a score: the values and a flag, 80 KB at the limit).
+constexpr int kSmallN = 16384;
 // Largest k the radix path handles (its final sort holds k positions in smem).
 constexpr int kLargeMaxK = 16384;
 

@@ -17,7 +17,8 @@ def _run(rba, s, k, base=0):
 
 @pytest.mark.parametrize("n,k,ties", [(1, 1, 0), (2, 1, 0), (61, 4, 0), (991, 32, 0),
                                       (991, 32, 5), (1000, 1000, 3), (4096, 4096, 0),
-                                      (8192, 100, 2), (5000, 1, 0), (7, 7, 1)])
+                                      (8192, 100, 2), (5000, 1, 0), (7, 7, 1),
+                                      (8193, 2048, 0), (16383, 256, 3), (16384, 2048, 0)])
 def test_topk_small_rows(rba, n, k, ties):
     s = synth.random_scores(20 + n + k, 6, n, ties=ties)
     got = _run(rba, s, k, base=3)
@@ -25,8 +26,8 @@ def test_topk_small_rows(rba, n, k, ties):
         np.testing.assert_array_equal(got[r], O.top_k(s[r].astype(np.float64), k) + 3)
 
 
-@pytest.mark.parametrize("n,k,ties", [(8193, 2048, 0), (65536, 256, 0), (1 << 20, 2048, 0),
-                                      (100000, 2048, 4), (50000, 16384, 0), (9000, 9000, 0)])
+@pytest.mark.parametrize("n,k,ties", [(16385, 2048, 0), (65536, 256, 0), (1 << 20, 2048, 0),
+                                      (100000, 2048, 4), (50000, 16384, 0), (16400, 16384, 0)])
 def test_topk_large_rows(rba, n, k, ties):
     s = synth.random_scores(7 + k, 3, n, ties=ties)
     got = _run(rba, s, k)
