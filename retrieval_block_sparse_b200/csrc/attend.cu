@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1) attend_decode_kernel(Attend
   const int split = blockIdx.x, bh = blockIdx.y;
   const int nseg = a.k + 2;
   const int n_att = build_segments(a, bh, sstart, svstart, s_warp);
+  // token-level retrieval with every selected token in place: direct mapping
+  const bool unit = a.bs == 1 && svstart[nseg - 1] == svstart[1] + a.k;
   const int v_lo = static_cast<int>(int64_t(n_att) * split / a.nsplit);
   const int v_hi = static_cast<int>(int64_t(n_att) * (split + 1) / a.nsplit);
   const int ntiles = (v_hi - v_lo + C::TT - 1) / C::TT;
@@ -39,14 +41,14 @@ __global__ void __launch_bounds__(kAttendThreads, 1) attend_decode_kernel(Attend
   for (int s = 0; s < C::NS - 1; ++s) {
     if (s < ntiles)
       issue_tile<T, D>(a, row0, stages + s * C::STAGE, sstart, svstart, nseg, v_lo + s * C::TT,
-                       v_hi);
+                       v_hi, unit);
     cp_async_commit();
   }
   for (int t = 0; t < ntiles; ++t) {
     const int tn = t + C::NS - 1;
     if (tn < ntiles)
       issue_tile<T, D>(a, row0, stages + (tn % C::NS) * C::STAGE, sstart, svstart, nseg,
-                       v_lo + tn * C::TT, v_hi);
+                       v_lo + tn * C::TT, v_hi, unit);
     cp_async_commit();
     cp_async_wait<C::NS - 1>();
     __syncthreads();

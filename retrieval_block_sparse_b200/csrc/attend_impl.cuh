@@ -124,8 +124,15 @@ __device__ inline int build_segments(const AttendArgs& a, int bh, int* sstart, i
   return total;
 }
 
-// physical token of virtual position v (0 <= v < n_att)
-__device__ __forceinline__ int seg_map(const int* sstart, const int* svstart, int nseg, int v) {
+// physical token of virtual position v (0 <= v < n_att).  unit: every
+// selected segment is one token (token-level retrieval), so segment i >= 1
+// starts at virtual position svstart[1] + i - 1 and no search is needed.
+__device__ __forceinline__ int seg_map(const int* sstart, const int* svstart, int nseg, int v,
+                                       bool unit) {
+  if (unit) {
+    const int i = v < svstart[1] ? 0 : min(1 + v - svstart[1], nseg - 1);
+    return sstart[i] + (v - svstart[i]);
+  }
   int lo = 0, hi = nseg - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -140,7 +147,7 @@ __device__ __forceinline__ int seg_map(const int* sstart, const int* svstart, in
 template <typename T, int D>
 __device__ __forceinline__ void issue_tile(const AttendArgs& a, int64_t bh_row0, char* stage,
                                            const int* sstart, const int* svstart, int nseg,
-                                           int v0, int v1) {
+                                           int v0, int v1, bool unit) {
   using C = DecodeTile<T, D>;
   const char* Kb = static_cast<const char*>(a.K);
   const char* Vb = static_cast<const char*>(a.V);
@@ -153,7 +160,7 @@ __device__ __forceinline__ void issue_tile(const AttendArgs& a, int64_t bh_row0,
     const int row = cc / C::CPR, col = cc % C::CPR;
     const int v = v0 + row;
     if (v < v1) {
-      const int64_t tok = bh_row0 + seg_map(sstart, svstart, nseg, v);
+      const int64_t tok = bh_row0 + seg_map(sstart, svstart, nseg, v, unit);
       const char* src = (isv ? Vb : Kb) + tok * C::ROWB + col * 16;
       cp_async16(stage + (isv ? HALF * 16 : 0) + row * C::ROWB + col * 16, src);
     }
