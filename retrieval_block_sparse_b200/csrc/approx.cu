@@ -48,9 +48,29 @@ __global__ void __launch_bounds__(128) stage2_kernel(const T* __restrict__ K,
   constexpr int EPV = Elem<T>::kPerVec;
   constexpr int LPT = D / EPV;
   constexpr int TPW = 32 / LPT;
+  constexpr int U = 8;  // key loads in flight per lane
   __shared__ float qs[D];
   const int gi = blockIdx.x, bh = blockIdx.y;
   const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  const int sub = lane % LPT;
+  const int stride = nwarp * TPW;  // tokens per load round of the CTA
+  const int64_t t0 = int64_t(kept[int64_t(bh) * C + gi]) * group;
+  const uint4* kb = reinterpret_cast<const uint4*>(K + int64_t(bh) * cap * D);
+  float* out = scores2 + (int64_t(bh) * C + gi) * group;
+  // this lane's token of load u of a batch: base + u * stride + (its slot)
+  const int slot = warp * TPW + lane / LPT;
+  uint4 kv[U];
+  auto load_batch = [&](int base) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int tt = base + u * stride + slot;
+      kv[u] = tt < group ? ld_stream(kb + (t0 + tt) * LPT + sub) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  // the first batch's loads are issued before the query is summed: the two
+  // latencies overlap
+  load_batch(0);
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float acc = 0.f;  // (q rows are qd long; the pools' padding columns score zero)
     if (d < qd)
@@ -58,28 +78,24 @@ __global__ void __launch_bounds__(128) stage2_kernel(const T* __restrict__ K,
     qs[d] = acc;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-  const int sub = lane % LPT;
   float qv[EPV];
 #pragma unroll
   for (int e = 0; e < EPV; ++e) qv[e] = qs[sub * EPV + e];
-  const int64_t t0 = int64_t(kept[int64_t(bh) * C + gi]) * group;
-  const uint4* kb = reinterpret_cast<const uint4*>(K + int64_t(bh) * cap * D);
-  float* out = scores2 + (int64_t(bh) * C + gi) * group;
-  for (int base = warp * TPW; base < group; base += nwarp * TPW) {
-    const int tt = base + lane / LPT;
-    const bool in = tt < group;
-    float part = 0.f;
-    if (in) {
+  for (int base = 0; base < group; base += U * stride) {
+    if (base > 0) load_batch(base);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int tt = base + u * stride + slot;
       float f[EPV];
-      unpack(ld_stream(kb + (t0 + tt) * LPT + sub), f, T());
+      unpack(kv[u], f, T());
+      float part = 0.f;
 #pragma unroll
       for (int e = 0; e < EPV; ++e) part = fmaf(qv[e], f[e], part);
-    }
 #pragma unroll
-    for (int o = LPT / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    const int64_t tok = t0 + tt;
-    if (in && sub == 0) out[tt] = tok >= sink && tok < w0 ? part : -INFINITY;
+      for (int o = LPT / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      const int64_t tok = t0 + tt;
+      if (tt < group && sub == 0) out[tt] = tok >= sink && tok < w0 ? part : -INFINITY;
+    }
   }
 }
 
