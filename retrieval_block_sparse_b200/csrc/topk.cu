@@ -136,13 +136,37 @@ __device__ bool select_binned(const float* s, int n, int k, int index_base, int3
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float lo = INFINITY, hi = -INFINITY;
   int bad = 0;
+  // long rows: sixteen loads in flight per thread before any store (two
+  // rounds at the longest rows instead of one per four scores); short rows
+  // (the decode step's) keep the plain loop
+  constexpr int kBatch = 16;
+  if (n <= 8 * kRowThreads) {
 #pragma unroll 4
-  for (int j = tid; j < n; j += kRowThreads) {
-    const float v = s[j];
-    vals[j] = v;
-    bad |= !isfinite(v);
-    lo = fminf(lo, v);
-    hi = fmaxf(hi, v);
+    for (int j = tid; j < n; j += kRowThreads) {
+      const float v = s[j];
+      vals[j] = v;
+      bad |= !isfinite(v);
+      lo = fminf(lo, v);
+      hi = fmaxf(hi, v);
+    }
+  }
+  for (int j0 = n <= 8 * kRowThreads ? n : tid; j0 < n; j0 += kBatch * kRowThreads) {
+    float v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = j0 + u * kRowThreads;
+      v[u] = j < n ? s[j] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = j0 + u * kRowThreads;
+      if (j < n) {
+        vals[j] = v[u];
+        bad |= !isfinite(v[u]);
+        lo = fminf(lo, v[u]);
+        hi = fmaxf(hi, v[u]);
+      }
+    }
   }
   for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0;
   for (int o = 16; o > 0; o >>= 1) {
