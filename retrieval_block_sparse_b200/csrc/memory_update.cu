@@ -9,6 +9,7 @@
 //                           threshold on the 32-bit counts, then an ordered scan
 //                           that writes the keep map (destination -> source block)
 //   memory_move_kernel      in-place compaction, one launch per round of destinations
+//                           (a CTA copies 32 KB of one block, 8 loads in flight a thread)
 //   memory_finish_kernel    moves the partial tail block, zeroes vacated counters
 //
 // In-place safety.  The keep map is strictly increasing and every kept entry
@@ -26,6 +27,9 @@ namespace {
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kMoveThreads = 256;
+constexpr int kMoveVecs = 8;                           // 16-byte loads in flight per thread
+constexpr int kChunkVecs = kMoveThreads * kMoveVecs;   // vectors a CTA copies (32 KB)
+constexpr int64_t kMaxMoveCtas = int64_t(1) << 30;      // K/V CTAs of one launch
 
 int grid_cap(int64_t work, int threads) {
   int64_t g = (work + threads - 1) / threads;
@@ -169,35 +173,52 @@ __device__ __forceinline__ bool source_ok(const MoveArgs& a, int32_t src, int32_
 }
 
 // Moves destinations [t0, t0 + nt) of every unit (see the safety note above).
+// A K/V row is one (unit, destination, head, K or V) block: bs * row_vecs
+// contiguous 16-byte vectors at both ends.  CTAs [0, kv_ctas) copy the rows,
+// `chunks` CTAs a row, each thread holding kMoveVecs loads in flight before
+// its stores; the remaining CTAs copy the per-block words (representation,
+// positions, counter).  All index arithmetic is once per CTA, in 32 bits.
 __global__ void __launch_bounds__(kMoveThreads)
-    memory_move_kernel(MoveArgs a, int32_t t0, int32_t nt) {
-  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  const int64_t first = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t blk_vecs = int64_t(a.bs) * a.row_vecs;
-  const int64_t total = int64_t(a.units) * nt * a.heads * 2 * blk_vecs;
-  for (int64_t i = first; i < total; i += stride) {
-    int64_t r = i / blk_vecs;
-    const int64_t e = i - r * blk_vecs;
-    const int kv = static_cast<int>(r & 1);
-    r >>= 1;
-    const int64_t h = r % a.heads;
-    r /= a.heads;
-    const int32_t t = t0 + static_cast<int32_t>(r % nt);
-    const int64_t u = r / nt;
-    const int32_t src = a.keep_map[u * a.keep_total + t];
+    memory_move_kernel(MoveArgs a, int32_t t0, int32_t nt, int32_t chunks, int32_t kv_ctas) {
+  const int tid = threadIdx.x;
+  if (static_cast<int32_t>(blockIdx.x) < kv_ctas) {
+    const uint32_t row = blockIdx.x / static_cast<uint32_t>(chunks);
+    const uint32_t chunk = blockIdx.x - row * static_cast<uint32_t>(chunks);
+    const uint32_t kv = row & 1u;
+    const uint32_t r = row >> 1;
+    const uint32_t uh = r / static_cast<uint32_t>(a.heads);  // unit * nt + (t - t0)
+    const uint32_t h = r - uh * static_cast<uint32_t>(a.heads);
+    const uint32_t u = uh / static_cast<uint32_t>(nt);
+    const int32_t t = t0 + static_cast<int32_t>(uh - u * static_cast<uint32_t>(nt));
+    const int32_t src = a.keep_map[int64_t(u) * a.keep_total + t];
     const int32_t dst = a.pinned + t;
-    if (src == dst || !source_ok(a, src, dst)) continue;
+    if (src == dst || !source_ok(a, src, dst)) return;
     uint4* pool = kv ? a.v : a.k;
-    const int64_t row0 = (u * a.heads + h) * a.cap_tokens;
-    pool[(row0 + int64_t(dst) * a.bs) * a.row_vecs + e] =
-        pool[(row0 + int64_t(src) * a.bs) * a.row_vecs + e];
+    const int64_t row0 = (int64_t(u) * a.heads + h) * a.cap_tokens;
+    const uint4* from = pool + (row0 + int64_t(src) * a.bs) * a.row_vecs;
+    uint4* to = pool + (row0 + int64_t(dst) * a.bs) * a.row_vecs;
+    const int32_t blk_vecs = a.bs * a.row_vecs;
+    const int32_t e0 = static_cast<int32_t>(chunk) * kChunkVecs + tid;
+    uint4 v[kMoveVecs];
+#pragma unroll
+    for (int j = 0; j < kMoveVecs; ++j) {
+      const int32_t e = e0 + j * kMoveThreads;
+      if (e < blk_vecs) v[j] = ld_stream(from + e);
+    }
+#pragma unroll
+    for (int j = 0; j < kMoveVecs; ++j) {
+      const int32_t e = e0 + j * kMoveThreads;
+      if (e < blk_vecs) to[e] = v[j];
+    }
+    return;
   }
   // per-block words: representation, positions, counter
-  const int64_t words = int64_t(a.rep_words) + a.pos_words + 1;
-  const int64_t total2 = int64_t(a.units) * nt * words;
-  for (int64_t i = first; i < total2; i += stride) {
+  const int32_t words = a.rep_words + a.pos_words + 1;
+  const int64_t total = int64_t(a.units) * nt * words;
+  const int64_t stride = int64_t(gridDim.x - kv_ctas) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x - kv_ctas) * blockDim.x + tid; i < total; i += stride) {
     const int64_t r = i / words;
-    const int64_t w = i - r * words;
+    const int32_t w = static_cast<int32_t>(i - r * words);
     const int32_t t = t0 + static_cast<int32_t>(r % nt);
     const int64_t u = r / nt;
     const int32_t src = a.keep_map[u * a.keep_total + t];
@@ -207,7 +228,7 @@ __global__ void __launch_bounds__(kMoveThreads)
     if (w < a.rep_words) {
       a.rep[(b0 + dst) * a.rep_words + w] = a.rep[(b0 + src) * a.rep_words + w];
     } else if (w < a.rep_words + a.pos_words) {
-      const int64_t p = w - a.rep_words;
+      const int32_t p = w - a.rep_words;
       a.rep_pos[(b0 + dst) * a.pos_words + p] = a.rep_pos[(b0 + src) * a.pos_words + p];
     } else {
       a.counters[b0 + dst] = a.counters[b0 + src];
@@ -341,17 +362,30 @@ extern "C" rba_status rba_memory_update(rba_store* st, int64_t T, int32_t pinned
         static_cast<int32_t>(kk), static_cast<int32_t>(hi), static_cast<int32_t>(keep_newest),
         static_cast<int32_t>(keep_total), keep_map);
     RBA_LAUNCH_CHECK();
-    // rounds of g destinations; every kept entry moves by at least drop_oldest blocks
+    // rounds of g destinations; every kept entry moves by at least drop_oldest blocks.
+    // A round may be cut into several launches: each moves a subset of the
+    // round's destinations, whose sources none of them writes.
     const int64_t g = drop_oldest > 0 ? drop_oldest : 1;
-    const int64_t per_dest = int64_t(a.heads) * 2 * bs * a.row_vecs;
+    const int64_t blk_vecs = bs * a.row_vecs;
+    if (blk_vecs > INT32_MAX - kChunkVecs) return RBA_ERR_UNSUPPORTED;
+    const int64_t chunks = (blk_vecs + kChunkVecs - 1) / kChunkVecs;
+    const int64_t ctas_per_dest = int64_t(units) * a.heads * 2 * chunks;
+    if (ctas_per_dest > kMaxMoveCtas) return RBA_ERR_UNSUPPORTED;
+    const int64_t max_nt = kMaxMoveCtas / ctas_per_dest;
+    const int64_t words = a.rep_words + a.pos_words + 1;
     for (int64_t t0 = 0; t0 < keep_total; t0 += g) {
-      const int64_t nt = keep_total - t0 < g ? keep_total - t0 : g;
-      const int64_t work = units * nt * (per_dest > a.rep_words + a.pos_words + 1
-                                             ? per_dest
-                                             : a.rep_words + a.pos_words + 1);
-      memory_move_kernel<<<grid_cap(work, kMoveThreads), kMoveThreads, 0, stream>>>(
-          a, static_cast<int32_t>(t0), static_cast<int32_t>(nt));
-      RBA_LAUNCH_CHECK();
+      const int64_t round_end = t0 + g < keep_total ? t0 + g : keep_total;
+      for (int64_t s0 = t0; s0 < round_end; s0 += max_nt) {
+        const int64_t nt = round_end - s0 < max_nt ? round_end - s0 : max_nt;
+        const int64_t kv_ctas = nt * ctas_per_dest;
+        int64_t word_ctas = (int64_t(units) * nt * words + kMoveThreads - 1) / kMoveThreads;
+        if (word_ctas > num_sms()) word_ctas = num_sms();
+        memory_move_kernel<<<static_cast<unsigned>(kv_ctas + word_ctas), kMoveThreads, 0,
+                             stream>>>(a, static_cast<int32_t>(s0), static_cast<int32_t>(nt),
+                                       static_cast<int32_t>(chunks),
+                                       static_cast<int32_t>(kv_ctas));
+        RBA_LAUNCH_CHECK();
+      }
     }
   }
   const int64_t clear_to = nb + 1 < st->cap_blocks ? nb + 1 : st->cap_blocks;
