@@ -8,7 +8,8 @@
 //   memory_select_kernel    one CTA per memory unit: radix select of the keep
 //                           threshold on the 32-bit counts, then an ordered scan
 //                           that writes the keep map (destination -> source block)
-//   memory_move_kernel      in-place compaction, one launch per round of destinations
+//   memory_move_kernel      in-place compaction, one launch per round of destinations,
+//                           each a programmatic dependent of the kernel before it
 //                           (a CTA copies 32 KB of one block, 8 loads in flight a thread)
 //   memory_finish_kernel    moves the partial tail block, zeroes vacated counters
 //
@@ -27,7 +28,8 @@ namespace {
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kMoveThreads = 256;
-constexpr int kMoveVecs = 8;                           // 16-byte loads in flight per thread
+constexpr int kMoveWarps = kMoveThreads / 32;
+constexpr int kMoveVecs = 8;                           // loads in flight per thread
 constexpr int kChunkVecs = kMoveThreads * kMoveVecs;   // vectors a CTA copies (32 KB)
 constexpr int64_t kMaxMoveCtas = int64_t(1) << 30;      // K/V CTAs of one launch
 
@@ -83,6 +85,8 @@ __global__ void __launch_bounds__(kSelThreads)
   __shared__ uint32_t hist[256];
   __shared__ uint32_t swarp[kSelWarps];
   __shared__ uint32_t s_digit, s_rem;
+  // the first move kernel may become resident now (it waits for our completion)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x;
   const uint32_t* cnt = counters + int64_t(blockIdx.x) * cap_blocks + lo;
   int32_t* map = keep_map + int64_t(blockIdx.x) * keep_total;
@@ -92,8 +96,24 @@ __global__ void __launch_bounds__(kSelThreads)
   const bool keep_none = kk == 0, keep_all = kk == mid;
   uint32_t thr = 0, need = 0, n_eq = 0;
   if (!keep_none && !keep_all) {
+    // digits above the largest count's top digit are zero for every entry:
+    // the select starts at that digit
+    uint32_t cmax = 0;
+    for (int64_t i = tid; i < mid; i += kSelThreads) cmax = max(cmax, cnt[i]);
+    cmax = __reduce_max_sync(0xffffffffu, cmax);
+    if ((tid & 31) == 0) swarp[tid >> 5] = cmax;
+    __syncthreads();
+    if (tid < 32) {
+      uint32_t m = tid < kSelWarps ? swarp[tid] : 0u;
+      m = __reduce_max_sync(0xffffffffu, m);
+      if (tid == 0) s_digit = m;
+    }
+    __syncthreads();
+    cmax = s_digit;
+    int top = 0;
+    while (top < 24 && (cmax >> (top + 8)) != 0u) top += 8;
     uint32_t prefix = 0, mask = 0, rem = static_cast<uint32_t>(kk);
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int shift = top; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
       __syncthreads();
       for (int64_t base = 0; base < mid; base += kSelThreads) {
@@ -104,15 +124,43 @@ __global__ void __launch_bounds__(kSelThreads)
         if (bin < 256 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
       }
       __syncthreads();
-      if (tid == 0) {  // highest digit whose bucket holds the rem-th largest
-        uint32_t above = 0;
-        int d = 255;
-        for (; d > 0; --d) {
-          if (above + hist[d] >= rem) break;
-          above += hist[d];
+      if (tid < 32) {
+        // the highest digit d >= 1 whose suffix count S(d) = sum_{i >= d} hist[i]
+        // reaches rem (else 0); lane l holds bins [8 l, 8 l + 8)
+        uint32_t h8[8], own = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          h8[b] = hist[tid * 8 + b];
+          own += h8[b];
         }
-        s_digit = static_cast<uint32_t>(d);
-        s_rem = rem - above;
+        uint32_t incl = own;  // sum over lanes >= tid
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
+          if (tid + o < 32) incl += y;
+        }
+        uint32_t suf = incl - own;  // S(8 tid + 8)
+        int found = -1;
+        uint32_t above = 0;
+#pragma unroll
+        for (int b = 7; b >= 0; --b) {
+          const int d = tid * 8 + b;
+          if (found < 0 && d >= 1 && suf + h8[b] >= rem) {
+            found = d;
+            above = suf;
+          }
+          suf += h8[b];
+        }
+        const unsigned hits = __ballot_sync(0xffffffffu, found >= 0);
+        if (hits == 0u) {
+          if (tid == 0) {  // digit 0: every entry of bins 1..255 is above
+            s_digit = 0;
+            s_rem = rem - (incl - h8[0]);
+          }
+        } else if (tid == 31 - __clz(hits)) {
+          s_digit = static_cast<uint32_t>(found);
+          s_rem = rem - above;
+        }
       }
       __syncthreads();
       prefix |= s_digit << shift;
@@ -172,67 +220,86 @@ __device__ __forceinline__ bool source_ok(const MoveArgs& a, int32_t src, int32_
   return false;
 }
 
+// Launched as a programmatic dependent of the previous kernel of the update:
+// it may become resident early, but touches no memory before that kernel has
+// completed; it lets the next kernel do the same.
+__device__ __forceinline__ void chain_entry() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Moves destinations [t0, t0 + nt) of every unit (see the safety note above).
-// A K/V row is one (unit, destination, head, K or V) block: bs * row_vecs
-// contiguous 16-byte vectors at both ends.  CTAs [0, kv_ctas) copy the rows,
-// `chunks` CTAs a row, each thread holding kMoveVecs loads in flight before
-// its stores; the remaining CTAs copy the per-block words (representation,
-// positions, counter).  All index arithmetic is once per CTA, in 32 bits.
+// CTAs [0, word_ctas) come first (scheduled first, so they are not a round's
+// tail): warp w of CTA b copies the per-block words of destination 8 b + w
+// (representation, positions, counter), kMoveVecs loads in flight a lane.
+// The other CTAs copy K/V rows: a row is one (unit, destination, head, K or
+// V) block, bs * row_vecs contiguous 16-byte vectors at both ends, `chunks`
+// CTAs a row, each thread holding kMoveVecs loads in flight before its stores.
+// All index arithmetic is once per CTA or warp, in 32 bits.
 __global__ void __launch_bounds__(kMoveThreads)
-    memory_move_kernel(MoveArgs a, int32_t t0, int32_t nt, int32_t chunks, int32_t kv_ctas) {
+    memory_move_kernel(MoveArgs a, int32_t t0, int32_t nt, int32_t chunks, int32_t word_ctas) {
+  chain_entry();
   const int tid = threadIdx.x;
-  if (static_cast<int32_t>(blockIdx.x) < kv_ctas) {
-    const uint32_t row = blockIdx.x / static_cast<uint32_t>(chunks);
-    const uint32_t chunk = blockIdx.x - row * static_cast<uint32_t>(chunks);
-    const uint32_t kv = row & 1u;
-    const uint32_t r = row >> 1;
-    const uint32_t uh = r / static_cast<uint32_t>(a.heads);  // unit * nt + (t - t0)
-    const uint32_t h = r - uh * static_cast<uint32_t>(a.heads);
-    const uint32_t u = uh / static_cast<uint32_t>(nt);
-    const int32_t t = t0 + static_cast<int32_t>(uh - u * static_cast<uint32_t>(nt));
+  if (static_cast<int32_t>(blockIdx.x) < word_ctas) {
+    const int lane = tid & 31;
+    const uint32_t di = blockIdx.x * kMoveWarps + (tid >> 5);
+    if (di >= static_cast<uint32_t>(a.units) * static_cast<uint32_t>(nt)) return;
+    const uint32_t u = di / static_cast<uint32_t>(nt);
+    const int32_t t = t0 + static_cast<int32_t>(di - u * static_cast<uint32_t>(nt));
     const int32_t src = a.keep_map[int64_t(u) * a.keep_total + t];
     const int32_t dst = a.pinned + t;
     if (src == dst || !source_ok(a, src, dst)) return;
-    uint4* pool = kv ? a.v : a.k;
-    const int64_t row0 = (int64_t(u) * a.heads + h) * a.cap_tokens;
-    const uint4* from = pool + (row0 + int64_t(src) * a.bs) * a.row_vecs;
-    uint4* to = pool + (row0 + int64_t(dst) * a.bs) * a.row_vecs;
-    const int32_t blk_vecs = a.bs * a.row_vecs;
-    const int32_t e0 = static_cast<int32_t>(chunk) * kChunkVecs + tid;
-    uint4 v[kMoveVecs];
+    const int64_t b0 = int64_t(u) * a.cap_blocks;
+    if (a.rep_words > 0) {
+      const uint32_t* from = a.rep + (b0 + src) * a.rep_words;
+      uint32_t* to = a.rep + (b0 + dst) * a.rep_words;
+      for (int32_t base = 0; base < a.rep_words; base += 32 * kMoveVecs) {
+        uint32_t w[kMoveVecs];
 #pragma unroll
-    for (int j = 0; j < kMoveVecs; ++j) {
-      const int32_t e = e0 + j * kMoveThreads;
-      if (e < blk_vecs) v[j] = ld_stream(from + e);
-    }
+        for (int j = 0; j < kMoveVecs; ++j) {
+          const int32_t i = base + j * 32 + lane;
+          if (i < a.rep_words) w[j] = from[i];
+        }
 #pragma unroll
-    for (int j = 0; j < kMoveVecs; ++j) {
-      const int32_t e = e0 + j * kMoveThreads;
-      if (e < blk_vecs) to[e] = v[j];
+        for (int j = 0; j < kMoveVecs; ++j) {
+          const int32_t i = base + j * 32 + lane;
+          if (i < a.rep_words) to[i] = w[j];
+        }
+      }
     }
+    for (int32_t i = lane; i < a.pos_words; i += 32)
+      a.rep_pos[(b0 + dst) * a.pos_words + i] = a.rep_pos[(b0 + src) * a.pos_words + i];
+    if (lane == 0) a.counters[b0 + dst] = a.counters[b0 + src];
     return;
   }
-  // per-block words: representation, positions, counter
-  const int32_t words = a.rep_words + a.pos_words + 1;
-  const int64_t total = int64_t(a.units) * nt * words;
-  const int64_t stride = int64_t(gridDim.x - kv_ctas) * blockDim.x;
-  for (int64_t i = int64_t(blockIdx.x - kv_ctas) * blockDim.x + tid; i < total; i += stride) {
-    const int64_t r = i / words;
-    const int32_t w = static_cast<int32_t>(i - r * words);
-    const int32_t t = t0 + static_cast<int32_t>(r % nt);
-    const int64_t u = r / nt;
-    const int32_t src = a.keep_map[u * a.keep_total + t];
-    const int32_t dst = a.pinned + t;
-    if (src == dst || !source_ok(a, src, dst)) continue;
-    const int64_t b0 = u * a.cap_blocks;
-    if (w < a.rep_words) {
-      a.rep[(b0 + dst) * a.rep_words + w] = a.rep[(b0 + src) * a.rep_words + w];
-    } else if (w < a.rep_words + a.pos_words) {
-      const int32_t p = w - a.rep_words;
-      a.rep_pos[(b0 + dst) * a.pos_words + p] = a.rep_pos[(b0 + src) * a.pos_words + p];
-    } else {
-      a.counters[b0 + dst] = a.counters[b0 + src];
-    }
+  const uint32_t row = (blockIdx.x - static_cast<uint32_t>(word_ctas)) / static_cast<uint32_t>(chunks);
+  const uint32_t chunk =
+      blockIdx.x - static_cast<uint32_t>(word_ctas) - row * static_cast<uint32_t>(chunks);
+  const uint32_t kv = row & 1u;
+  const uint32_t r = row >> 1;
+  const uint32_t uh = r / static_cast<uint32_t>(a.heads);  // unit * nt + (t - t0)
+  const uint32_t h = r - uh * static_cast<uint32_t>(a.heads);
+  const uint32_t u = uh / static_cast<uint32_t>(nt);
+  const int32_t t = t0 + static_cast<int32_t>(uh - u * static_cast<uint32_t>(nt));
+  const int32_t src = a.keep_map[int64_t(u) * a.keep_total + t];
+  const int32_t dst = a.pinned + t;
+  if (src == dst || !source_ok(a, src, dst)) return;
+  uint4* pool = kv ? a.v : a.k;
+  const int64_t row0 = (int64_t(u) * a.heads + h) * a.cap_tokens;
+  const uint4* from = pool + (row0 + int64_t(src) * a.bs) * a.row_vecs;
+  uint4* to = pool + (row0 + int64_t(dst) * a.bs) * a.row_vecs;
+  const int32_t blk_vecs = a.bs * a.row_vecs;
+  const int32_t e0 = static_cast<int32_t>(chunk) * kChunkVecs + tid;
+  uint4 v[kMoveVecs];
+#pragma unroll
+  for (int j = 0; j < kMoveVecs; ++j) {
+    const int32_t e = e0 + j * kMoveThreads;
+    if (e < blk_vecs) v[j] = ld_stream(from + e);
+  }
+#pragma unroll
+  for (int j = 0; j < kMoveVecs; ++j) {
+    const int32_t e = e0 + j * kMoveThreads;
+    if (e < blk_vecs) to[e] = v[j];
   }
 }
 
@@ -242,6 +309,7 @@ __global__ void __launch_bounds__(kMoveThreads)
 __global__ void __launch_bounds__(kMoveThreads)
     memory_finish_kernel(MoveArgs a, int32_t src_blk, int32_t dst_blk, int32_t tail,
                          int32_t clear_from, int32_t clear_to) {
+  chain_entry();
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
   const int64_t first = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t tail_vecs = int64_t(tail) * a.row_vecs;
@@ -261,6 +329,24 @@ __global__ void __launch_bounds__(kMoveThreads)
     const int64_t u = i / span;
     a.counters[u * a.cap_blocks + clear_from + (i - u * span)] = 0u;
   }
+}
+
+// Launches kernel (kMoveThreads threads) as a programmatic dependent of the
+// stream's previous kernel; the kernel begins with chain_entry().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, cudaStream_t stream,
+                           Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kMoveThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 int32_t units_of(const rba_store* st) {
@@ -372,19 +458,17 @@ extern "C" rba_status rba_memory_update(rba_store* st, int64_t T, int32_t pinned
     const int64_t ctas_per_dest = int64_t(units) * a.heads * 2 * chunks;
     if (ctas_per_dest > kMaxMoveCtas) return RBA_ERR_UNSUPPORTED;
     const int64_t max_nt = kMaxMoveCtas / ctas_per_dest;
-    const int64_t words = a.rep_words + a.pos_words + 1;
     for (int64_t t0 = 0; t0 < keep_total; t0 += g) {
       const int64_t round_end = t0 + g < keep_total ? t0 + g : keep_total;
       for (int64_t s0 = t0; s0 < round_end; s0 += max_nt) {
         const int64_t nt = round_end - s0 < max_nt ? round_end - s0 : max_nt;
-        const int64_t kv_ctas = nt * ctas_per_dest;
-        int64_t word_ctas = (int64_t(units) * nt * words + kMoveThreads - 1) / kMoveThreads;
-        if (word_ctas > num_sms()) word_ctas = num_sms();
-        memory_move_kernel<<<static_cast<unsigned>(kv_ctas + word_ctas), kMoveThreads, 0,
-                             stream>>>(a, static_cast<int32_t>(s0), static_cast<int32_t>(nt),
-                                       static_cast<int32_t>(chunks),
-                                       static_cast<int32_t>(kv_ctas));
-        RBA_LAUNCH_CHECK();
+        const int64_t word_ctas = (int64_t(units) * nt + kMoveWarps - 1) / kMoveWarps;
+        const int64_t ctas = nt * ctas_per_dest + word_ctas;
+        if (ctas > INT32_MAX) return RBA_ERR_UNSUPPORTED;
+        RBA_CUDA_TRY(launch_chained(memory_move_kernel, dim3(static_cast<unsigned>(ctas)), stream,
+                                    a, static_cast<int32_t>(s0), static_cast<int32_t>(nt),
+                                    static_cast<int32_t>(chunks),
+                                    static_cast<int32_t>(word_ctas)));
       }
     }
   }
@@ -393,11 +477,11 @@ extern "C" rba_status rba_memory_update(rba_store* st, int64_t T, int32_t pinned
   if (move_tail || clear_to > new_nb) {
     const int64_t work = units * a.heads * 2 * (move_tail ? tail : 0) * a.row_vecs +
                          units * (clear_to > new_nb ? clear_to - new_nb : 0);
-    memory_finish_kernel<<<grid_cap(work, kMoveThreads), kMoveThreads, 0, stream>>>(
-        a, static_cast<int32_t>(nb), static_cast<int32_t>(new_nb),
+    RBA_CUDA_TRY(launch_chained(
+        memory_finish_kernel, dim3(grid_cap(work, kMoveThreads)), stream, a,
+        static_cast<int32_t>(nb), static_cast<int32_t>(new_nb),
         static_cast<int32_t>(move_tail ? tail : 0), static_cast<int32_t>(new_nb),
-        static_cast<int32_t>(clear_to > new_nb ? clear_to : new_nb));
-    RBA_LAUNCH_CHECK();
+        static_cast<int32_t>(clear_to > new_nb ? clear_to : new_nb)));
   }
   return RBA_OK;
 }
