@@ -18,8 +18,9 @@
 // so each move spans at least g = drop_oldest blocks.  A round moves the
 // destinations [t0, t0 + g): it writes blocks [pinned + t0, pinned + t0 + g)
 // and reads blocks >= pinned + t0 + g, none of which a round writes before the
-// source has been read (later rounds read higher blocks still).  With
-// drop_oldest = 0 a round moves one entry.
+// source has been read (later rounds read higher blocks still); a round of
+// fewer destinations is safe all the more.  With drop_oldest = 0 a round
+// moves one entry.
 #include "rba_internal.cuh"
 
 namespace rba {
@@ -448,10 +449,13 @@ extern "C" rba_status rba_memory_update(rba_store* st, int64_t T, int32_t pinned
         static_cast<int32_t>(kk), static_cast<int32_t>(hi), static_cast<int32_t>(keep_newest),
         static_cast<int32_t>(keep_total), keep_map);
     RBA_LAUNCH_CHECK();
-    // rounds of g destinations; every kept entry moves by at least drop_oldest blocks.
-    // A round may be cut into several launches: each moves a subset of the
-    // round's destinations, whose sources none of them writes.
-    const int64_t g = drop_oldest > 0 ? drop_oldest : 1;
+    // rounds of at most drop_oldest destinations (every kept entry moves by at
+    // least that many blocks), as many as that takes and as even as possible
+    // (no short last round).  A round may be cut into several launches: each
+    // moves a subset of the round's destinations, whose sources none of them writes.
+    const int64_t g_max = drop_oldest > 0 ? drop_oldest : 1;
+    const int64_t n_rounds = (keep_total + g_max - 1) / g_max;
+    const int64_t g = n_rounds > 0 ? (keep_total + n_rounds - 1) / n_rounds : g_max;
     const int64_t blk_vecs = bs * a.row_vecs;
     if (blk_vecs > INT32_MAX - kChunkVecs) return RBA_ERR_UNSUPPORTED;
     const int64_t chunks = (blk_vecs + kChunkVecs - 1) / kChunkVecs;

@@ -224,3 +224,66 @@ def test_decode_count_update_decode_matches_oracle(rba):
         cnt = step(T_new, K2, V2, cnt)
     st.check()
     np.testing.assert_array_equal(counters.cpu().numpy().astype(np.int64), cnt)
+
+
+@pytest.mark.parametrize("name", ["infllm-decode-128k", "memlong-cosine-prefill"])
+def test_memory_update_full_size(rba, name):
+    """The update of the full 128K store (8 kv heads x 1023 blocks after the
+    sink) and of the full MemLong bank (160 chunks x 512 tokens x 32 heads),
+    with the counters, rule and launch configuration the bench times.  Keep
+    maps equal the oracle's memory_keep entry for entry; on sampled
+    destinations (the first and last three and 40 drawn at random per unit)
+    K, V, representation, positions and counter hold the bits of their source
+    block; vacated counters are zero and the pinned blocks are untouched."""
+    w = synth.WORKLOADS[name]
+    cosine = getattr(w, "score_mode", "dot") == "cosine"
+    if cosine:
+        mode, r, d_ret, batch = "embed_cosine", 1, w.d_ret, 1
+    else:
+        mode, r, d_ret, batch = w.rep_mode, w.n_rep, 0, w.batch
+    st = rba.Store(batch=batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                   head_dim=w.head_dim, block_size=w.block_size, capacity_tokens=w.context,
+                   dtype=w.dtype, mode=mode, n_rep=r, d_ret=d_ret)
+    gen = torch.Generator(device="cuda").manual_seed(w.seed)
+    for t in (st.k, st.v, st.rep):
+        if t is not None:
+            t.copy_(torch.randn(t.shape, generator=gen, device="cuda", dtype=torch.float32))
+    if st.rep_pos is not None:
+        st.rep_pos.random_(0, w.block_size, generator=gen)
+    U = st.memory_units()
+    counts = synth.retrieval_counts(w.seed, U, st.cap_blocks)
+    counters = torch.from_numpy(counts.view(np.int32)).cuda()
+    T, bs = w.context, w.block_size
+    nb = T // bs
+    pinned = -(-w.sink // bs) if w.sink else 0
+    newest, oldest, total = O.memory_rule(nb - pinned)
+    before = [t.clone() for t in (st.k, st.v, st.rep, st.rep_pos) if t is not None]
+    T_new, kmap = st.memory_update(T, counters, pinned_blocks=pinned)
+    st.check()
+    assert T_new == (pinned + total) * bs + (T - nb * bs)
+    kmap = kmap.cpu().numpy()
+    cnt1 = counters.cpu().numpy().view(np.uint32)
+    after = [t for t in (st.k, st.v, st.rep, st.rep_pos) if t is not None]
+    rng = np.random.default_rng(w.seed)
+    bits = lambda t: t.view(torch.int16) if t.dtype == torch.bfloat16 else t  # noqa: E731
+    for u in range(U):
+        keep = O.memory_keep(counts[u].astype(np.int64), nb, pinned, newest, oldest, total)
+        np.testing.assert_array_equal(kmap[u], keep)
+        sample = sorted(set([0, 1, 2, total - 3, total - 2, total - 1]) |
+                        set(rng.integers(0, total, 40).tolist()))
+        b, h = (u, slice(None)) if cosine else divmod(u, w.n_kv_heads)
+        for t in sample:
+            src, dst = int(keep[t]), pinned + t
+            for a0, a1 in zip(before[:2], after[:2]):  # K, V rows of the block
+                assert torch.equal(bits(a1[b, h, dst * bs:(dst + 1) * bs]),
+                                   bits(a0[b, h, src * bs:(src + 1) * bs])), (u, t)
+            for a0, a1 in zip(before[2:], after[2:]):  # representation, positions
+                ix = (b, dst) if cosine else (b, h, dst)
+                jx = (b, src) if cosine else (b, h, src)
+                assert torch.equal(bits(a1[ix]), bits(a0[jx])), (u, t)
+            assert cnt1[u, dst] == counts[u, src], (u, t)
+        assert not cnt1[u, pinned + total:nb].any()
+        for j in range(pinned):
+            for a0, a1 in zip(before[:2], after[:2]):
+                assert torch.equal(bits(a1[b, h, j * bs:(j + 1) * bs]),
+                                   bits(a0[b, h, j * bs:(j + 1) * bs]))
