@@ -244,7 +244,7 @@ rba_status rba_approx_select(const rba_store* st, const void* q, int64_t T, int3
   const ApproxWs w = approx_layout(workspace, BH, n_groups, groups_kept, group, k);
   if (workspace == nullptr || ws_bytes < w.total) return RBA_ERR_WORKSPACE;
   // stage 1: the candidate groups' means against the summed query, top groups_kept
-  ScoreArgs a;
+  ScoreArgs a = {};
   a.rep = means;
   a.rep_rows = d.capacity_tokens / group;
   a.q = q;

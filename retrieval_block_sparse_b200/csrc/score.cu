@@ -137,13 +137,14 @@ rba_status launch_qsum(const rba_store* st, const void* q, int n_q, float* qsum,
 
 // Dot-mode launch: templated on query, rep element type, head dim and rep count.
 rba_status launch_score_dot(const rba_store* st, const void* q, int n_q, const float* qsum,
-                            const Geometry& g, float* scores, cudaStream_t stream) {
+                            const Geometry& g, float* scores, cudaStream_t stream,
+                            int ctas_per_sm) {
   const rba_store_desc& d = st->d;
   const int BH = d.batch * d.n_kv_heads;
   const int grp = d.n_q_heads / d.n_kv_heads;
   if (qsum == nullptr && grp * n_q > 64) return RBA_ERR_INVALID_ARG;
   if (g.nc == 0) return RBA_OK;
-  ScoreArgs a;
+  ScoreArgs a = {};
   a.q = q;
   a.qsum = qsum;
   a.scores = scores;
@@ -154,6 +155,7 @@ rba_status launch_score_dot(const rba_store* st, const void* q, int n_q, const f
   a.nc = g.nc;
   a.qd = d.head_dim;
   a.max_over_keys = st->score_reduce == RBA_SCORE_MAX;
+  a.ctas_per_sm = ctas_per_sm;
   if (d.mode == RBA_REP_IDENTITY) {
     a.rep = st->k;
     a.rep_rows = d.capacity_tokens;

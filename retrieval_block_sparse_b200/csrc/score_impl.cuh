@@ -14,6 +14,7 @@ struct ScoreArgs {
   int Hq, Hkv, n_q, first, nc;
   int qd;               // row length of q (the rep rows hold D >= qd elements, the rest zero)
   bool max_over_keys;   // block score = max over its keys (else their sum)
+  int ctas_per_sm;      // grid target (host side): CTAs per SM
 };
 
 // One CTA covers `cand_per_cta` consecutive candidates of one (b, kv head).
@@ -142,7 +143,11 @@ rba_status launch_score_dot_t(const ScoreArgs& a, int BH, cudaStream_t stream) {
   constexpr int VPC = R * D / EPV;
   constexpr int LPC = VPC < 32 ? VPC : 32;
   constexpr int per_iter = NW * (32 / LPC) * U;
-  const int64_t want = int64_t(num_sms()) * 4;
+  // fewer than 4 CTAs per SM only where 4 would leave each CTA one batch of
+  // loads anyway (a short, latency-bound scan); long scans keep 4
+  int cps = a.ctas_per_sm > 0 ? a.ctas_per_sm : 4;
+  if (cps < 4 && int64_t(a.nc) * BH > int64_t(num_sms()) * 4 * per_iter) cps = 4;
+  const int64_t want = int64_t(num_sms()) * cps;
   int64_t per_cta = (int64_t(a.nc) * BH + want - 1) / want;
   per_cta = (per_cta + per_iter - 1) / per_iter * per_iter;
   if (per_cta < per_iter) per_cta = per_iter;
@@ -188,8 +193,12 @@ inline rba_status dispatch_score_dot(const ScoreArgs& a, bool q_bf16, bool rep_f
   return RBA_ERR_UNSUPPORTED;
 }
 
+// ctas_per_sm: the grid's target CTAs per SM (4 keeps enough loads in flight
+// for long scans; 1 leaves every SM room for a persistent kernel that starts
+// beside the score kernel as its programmatic dependent)
 rba_status launch_score_dot(const rba_store* st, const void* q, int n_q, const float* qsum,
-                            const Geometry& g, float* scores, cudaStream_t stream);
+                            const Geometry& g, float* scores, cudaStream_t stream,
+                            int ctas_per_sm = 4);
 rba_status launch_qsum(const rba_store* st, const void* q, int n_q, float* qsum,
                        cudaStream_t stream);
 
