@@ -307,9 +307,11 @@ rba_status rba_decode_step(const rba_store* st, const void* q, int32_t k, int64_
   // for their inputs on the device
   const bool fused = use_fused(st, g, k);
   if (k > 0) {
-    // before the persistent kernel: one score CTA per SM, so that every
-    // attention CTA fits beside one and starts streaming the sink/window rows
-    // while the scores are computed (1 CTA per SM: 128K step 21.5 -> 20.8 us)
+    // before the persistent kernel: at most one score CTA per SM, so that
+    // some SMs are empty from the start and the score CTAs retire together;
+    // the attention CTAs (which cannot share an SM with a score CTA: their
+    // registers fill an SM sub-partition) then start earlier and stream the
+    // sink/window rows while the top-k runs (128K step 21.5 -> 20.8 us)
     s = launch_score_dot(st, q, 1, nullptr, g, sc, stream, fused ? 1 : 4);
     if (s != RBA_OK) return s;
     s = launch_topk(sc, BH, g.nc, k, g.first, idx, w.topk_ws, w.topk_bytes, stream, fused);

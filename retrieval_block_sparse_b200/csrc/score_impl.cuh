@@ -194,8 +194,9 @@ inline rba_status dispatch_score_dot(const ScoreArgs& a, bool q_bf16, bool rep_f
 }
 
 // ctas_per_sm: the grid's target CTAs per SM (4 keeps enough loads in flight
-// for long scans; 1 leaves every SM room for a persistent kernel that starts
-// beside the score kernel as its programmatic dependent)
+// for long scans; 1, for short scans, leaves some SMs empty and lets the CTAs
+// retire together, so that a persistent kernel launched as a programmatic
+// dependent gets SMs sooner)
 rba_status launch_score_dot(const rba_store* st, const void* q, int n_q, const float* qsum,
                             const Geometry& g, float* scores, cudaStream_t stream,
                             int ctas_per_sm = 4);
