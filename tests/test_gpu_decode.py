@@ -148,3 +148,35 @@ def test_planted_blocks_retrieved_on_gpu(rba):
     hits = sum(len(set(idx[0, h]) & set(x["planted_blocks"][0, h])) for h in range(w.n_kv_heads))
     chance = w.n_kv_heads * w.n_planted * w.top_k / ref["cand"].shape[0]
     assert hits > 4 * chance
+
+
+@pytest.mark.parametrize("name", ["infllm-decode-128k", "landmark-decode-b16",
+                                  "token-retrieval-decode-1m", "ragged-f32"])
+def test_decode_step_host(rba, name):
+    """The step through rba_decode_step_host, the entry point the bench's
+    end-to-end figure uses: q from pinned host memory, out, lse and the
+    selection copied back to pinned host buffers, the call synchronising.
+    The host outputs are checked against the oracle as the device step's are,
+    on two calls over one workspace."""
+    w, x, reps, pos, ref = _prepared(name)
+    st = make_decode_store(rba, w, x)
+    q = dev(x["q"], w.dtype)
+    q_host = q.cpu().pin_memory()
+    B, Hq, Hkv, D = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim
+    q_dev = torch.empty_like(q)
+    idx_dev = torch.empty((B, Hkv, w.top_k), dtype=torch.int32, device="cuda")
+    out_dev = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+    lse_dev = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    out_h = torch.empty(out_dev.shape, dtype=torch.float32).pin_memory()
+    lse_h = torch.empty(lse_dev.shape, dtype=torch.float32).pin_memory()
+    idx_h = torch.empty(idx_dev.shape, dtype=torch.int32).pin_memory()
+    ws = st.decode_workspace(w.top_k, w.context, w.sink, w.window)
+    for _ in range(2):
+        out_h.fill_(float("nan"))
+        idx_h.fill_(-1)
+        st.decode_step_host(q_host, w.top_k, w.context, w.sink, w.window, q_dev=q_dev,
+                            idx_dev=idx_dev, out_dev=out_dev, lse_dev=lse_dev, out_host=out_h,
+                            lse_host=lse_h, idx_host=idx_h, workspace=ws)
+    st.check()
+    check_decode_step(w, x["q"], x["K"], x["V"], ref, idx_h.numpy(), out_h.numpy(),
+                      lse_h.numpy())
