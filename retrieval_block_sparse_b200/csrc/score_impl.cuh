@@ -136,18 +136,15 @@ __global__ void __launch_bounds__(NW * 32) score_dot_kernel(ScoreArgs a, int can
   }
 }
 
-template <typename QT, typename RT, int D, int R, bool MAXR>
-rba_status launch_score_dot_t(const ScoreArgs& a, int BH, cudaStream_t stream) {
-  constexpr int NW = 8, U = 4;
+// NW warps per CTA and U candidate groups in flight per warp; about `want`
+// CTAs in all (each warp at least one batch)
+template <int NW, int U, typename QT, typename RT, int D, int R, bool MAXR>
+rba_status launch_score_nw(const ScoreArgs& a, int BH, int64_t want, cudaStream_t stream) {
   constexpr int EPV = Elem<RT>::kPerVec;
   constexpr int VPC = R * D / EPV;
   constexpr int LPC = VPC < 32 ? VPC : 32;
   constexpr int per_iter = NW * (32 / LPC) * U;
-  // fewer than 4 CTAs per SM only where 4 would leave each CTA one batch of
-  // loads anyway (a short, latency-bound scan); long scans keep 4
-  int cps = a.ctas_per_sm > 0 ? a.ctas_per_sm : 4;
-  if (cps < 4 && int64_t(a.nc) * BH > int64_t(num_sms()) * 4 * per_iter) cps = 4;
-  const int64_t want = int64_t(num_sms()) * cps;
+  if (want < 1) want = 1;
   int64_t per_cta = (int64_t(a.nc) * BH + want - 1) / want;
   per_cta = (per_cta + per_iter - 1) / per_iter * per_iter;
   if (per_cta < per_iter) per_cta = per_iter;
@@ -156,6 +153,29 @@ rba_status launch_score_dot_t(const ScoreArgs& a, int BH, cudaStream_t stream) {
       <<<dim3(gx, BH), NW * 32, 0, stream>>>(a, static_cast<int>(per_cta));
   RBA_LAUNCH_CHECK();
   return RBA_OK;
+}
+
+template <typename QT, typename RT, int D, int R, bool MAXR>
+rba_status launch_score_dot_t(const ScoreArgs& a, int BH, cudaStream_t stream) {
+  constexpr int EPV = Elem<RT>::kPerVec;
+  constexpr int VPC = R * D / EPV;
+  constexpr int LPC = VPC < 32 ? VPC : 32;
+  constexpr int per_iter = 8 * (32 / LPC) * 4;  // candidates of one batch of an 8-warp CTA
+  // fewer than 4 CTAs per SM only where 4 would leave each CTA one batch of
+  // loads anyway (a short, latency-bound scan); long scans keep 4
+  int cps = a.ctas_per_sm > 0 ? a.ctas_per_sm : 4;
+  if (cps < 4 && int64_t(a.nc) * BH > int64_t(num_sms()) * 4 * per_iter) cps = 4;
+  // one CTA per SM: twice the candidate groups in flight per warp where a
+  // lane holds at most two vectors of a group (the registers are there with
+  // one CTA an SM; more vectors would spill), so that each warp's share is one
+  // batch of loads (128K step 20.83 -> 20.65 us)
+  if (cps == 1) {
+    if constexpr (VPC / LPC <= 2)
+      return launch_score_nw<8, 8, QT, RT, D, R, MAXR>(a, BH, num_sms(), stream);
+    else
+      return launch_score_nw<8, 4, QT, RT, D, R, MAXR>(a, BH, num_sms(), stream);
+  }
+  return launch_score_nw<8, 4, QT, RT, D, R, MAXR>(a, BH, int64_t(num_sms()) * cps, stream);
 }
 
 template <typename QT, typename RT, int D>
