@@ -448,9 +448,12 @@ rba_status rba_count_retrievals(const rba_store* store, const int32_t* idx, int3
  *             of the block now at pinned_blocks + t (may be NULL when keep_total = 0)
  * Requires 0 <= pinned_blocks <= nb, keep_newest + drop_oldest <= n and
  * keep_newest <= keep_total <= n - drop_oldest.  Launches one selection kernel,
- * ceil(keep_total / max(drop_oldest, 1)) move kernels (each moves entries that
- * are at least drop_oldest blocks from their destination, so no move overwrites
- * a block that is still to be read), and one kernel for the tail and counters.
+ * ceil(keep_total / max(drop_oldest, 1)) move kernels of as even a share of the
+ * destinations as possible (each moves entries that are at least drop_oldest
+ * blocks from their destination, so no move overwrites a block that is still to
+ * be read; a share too large for one grid is cut into several launches), and one
+ * kernel for the tail and counters; every kernel after the selection is a
+ * programmatic dependent of the one before it.
  * Errors: INVALID_ARG, UNSUPPORTED (nb >= 2^31 - 1), CUDA. */
 rba_status rba_memory_update(rba_store* store, int64_t T, int32_t pinned_blocks,
                              int64_t keep_newest, int64_t drop_oldest, int64_t keep_total,
